@@ -1,0 +1,450 @@
+"""Pins of the fp64 oracle to facts outside itself (CPU only).
+
+Each test ties the oracle to something the pages or the mathematics fix:
+closed forms printed on the pages, special cases with a textbook answer,
+invariants of softmax attention, and brute force on tiny inputs written
+independently with numpy/scipy. Together they are chosen so that a dropped
+term, a wrong sign, scale or index, an off-by-one mask or a transposed operand
+anywhere in the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from mla_latent_kv_18_b200.inputs import make_inputs, workload
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "cache_sizes.txt")
+
+# small variants of the five workloads (same head dims, fewer heads/tokens)
+SMALL = {
+    "tiny": workload("tiny", heads=4),
+    "dsv3": workload("dsv3", batch=2, heads=4, seq_len=200),
+    "ragged": workload("ragged", batch=3, heads=3, ragged=(65, 190)),
+    "retrofit": workload("retrofit", batch=2, heads=4, seq_len=130),
+}
+
+
+def _golden():
+    vals = {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = (s.strip() for s in line.split("="))
+                vals[k] = float(v)
+    return vals
+
+
+def _rel(a, b):
+    return np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300)
+
+
+def _bf16(x):
+    return torch.tensor(np.array(x, dtype=np.float64), dtype=torch.float32).to(torch.bfloat16)
+
+
+def _f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _dense_cache(inp):
+    """Logical (per-sequence, in token order) c_KV and k_R via numpy indexing."""
+    table = inp["block_table"].numpy()
+    lens = inp["seq_lens"].numpy()
+    ckv, kr = _f64(inp["ckv_pool"]), _f64(inp["kr_pool"])
+    P = ckv.shape[1]
+    out = []
+    for b, L in enumerate(lens):
+        t = np.arange(L)
+        pages = table[b, t // P]
+        out.append((ckv[pages, t % P], kr[pages, t % P]))
+    return out
+
+
+def _numpy_reference(inp, scale):
+    """Brute force: dense per-head keys/values, whole-row softmax (scipy)."""
+    qc, qr = _f64(inp["q_c"]), _f64(inp["q_r"])
+    wuk, wuv = _f64(inp["w_uk"]), _f64(inp["w_uv"])
+    B, n_q, H, _ = qc.shape
+    out = np.zeros((B, n_q, H, wuv.shape[-1]))
+    for b, (c, r) in enumerate(_dense_cache(inp)):
+        L = c.shape[0]
+        k_nope = np.einsum("sc,hdc->shd", c, wuk)          # path A of the page
+        v = np.einsum("sc,hce->she", c, wuv)
+        for i in range(n_q):
+            vis = L - n_q + i + 1
+            s = (np.einsum("hd,shd->hs", qc[b, i], k_nope[:vis])
+                 + np.einsum("hj,sj->hs", qr[b, i], r[:vis])) * scale
+            p = scipy.special.softmax(s, axis=-1)
+            out[b, i] = np.einsum("hs,she->he", p, v[:vis])
+    return out
+
+
+def _run_both(inp, scale=None):
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    dec = oracle.decode_decompress(*args, scale=scale)
+    ab, o_lat, lse = oracle.decode_absorbed(*args, scale=scale)
+    return dec, ab, o_lat, lse
+
+
+# ---------------------------------------------------------------------------
+# closed forms printed on the pages
+# ---------------------------------------------------------------------------
+
+def test_cache_size_closed_forms():
+    g = _golden()
+    assert 512 + 64 == g["mla_elements_per_token"]
+    assert 128 * 128 == g["mha_elements_per_head_block"]
+    assert oracle.mla_cache_bytes_per_token(512, 64) == g["mla_bytes_per_token"]
+    assert oracle.mla_cache_bytes_per_token(512, 64) / 1024 == 1.125
+    assert oracle.mha_cache_bytes_per_token(128, 128) == g["mha_bytes_per_token"]
+    comp = 100.0 * (1 - oracle.mla_cache_bytes_per_token(512, 64)
+                    / oracle.mha_cache_bytes_per_token(128, 128))
+    assert round(comp, 2) == g["compression_percent"]
+    tokens = g["total_context"] * g["total_batch"] * g["total_layers"]
+    mha = tokens * oracle.mha_cache_bytes_per_token(128, 128) / 2**40
+    gqa = tokens * oracle.mha_cache_bytes_per_token(8, 128) / 2**30
+    mla = tokens * oracle.mla_cache_bytes_per_token(512, 64) / 2**30
+    assert mha == pytest.approx(g["mha_total_tib"], rel=1e-12)
+    assert gqa == pytest.approx(g["gqa8_total_gib"], rel=0.03)
+    assert mla == pytest.approx(g["mla_total_gib"], rel=0.03)
+    # the latent page of 64 tokens is 72 KB ("MLA operator design" §3)
+    assert 64 * oracle.mla_cache_bytes_per_token(512, 64) == 72 * 1024
+    # "MHA2MLA" §4.2 formulas at its §3.2 dims
+    assert oracle.mha_cache_bytes_per_token(32, 128, 1) == g["retrofit_mha_elements_per_token"]
+    assert oracle.mla_cache_bytes_per_token(64, 8, 1) == g["retrofit_mla_elements_per_token"]
+
+
+def test_default_scale_is_page_value():
+    # scale = 1/sqrt(dhc + dr) with DeepSeek dims 128 + 64 ("MLA operator design" §4)
+    assert oracle.default_scale(128, 64) == 1.0 / math.sqrt(192.0)
+    assert oracle.default_scale(120, 8) == 1.0 / math.sqrt(128.0)
+
+
+# ---------------------------------------------------------------------------
+# P1 absorption identity and P4 brute force
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_absorption_identity_and_brute_force(name):
+    w = SMALL[name]
+    inp = make_inputs(w, seed=1)
+    dec, ab, o_lat, lse = _run_both(inp)
+    assert np.isfinite(dec).all()
+    assert _rel(ab, dec) <= 1e-12            # path A == path B (associativity)
+    ref = _numpy_reference(inp, oracle.default_scale(w.d_nope, w.d_rope))
+    assert _rel(dec, ref) <= 1e-12
+    assert np.abs(dec - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_sampled_selection_matches_full():
+    inp = make_inputs(SMALL["dsv3"], seed=2)
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    full = oracle.decode_decompress(*args)
+    sel = [1, 5, 6]
+    part = oracle.decode_decompress(*args, sel=sel)
+    flat_f, flat_p = full.reshape(-1, full.shape[-1]), part.reshape(-1, part.shape[-1])
+    np.testing.assert_array_equal(flat_p[sel], flat_f[sel])
+    assert not flat_p[0].any()
+
+
+# ---------------------------------------------------------------------------
+# special cases
+# ---------------------------------------------------------------------------
+
+def test_softmax_weights_sum_to_one():
+    # V[t] = c[t] W_UV with W_UV = identity and every c[t] = e_0  =>  out = (sum p) e_0
+    w = workload("dsv3", batch=2, heads=3, seq_len=150, d_latent=64, d_v=64)
+    inp = make_inputs(w, seed=3)
+    ckv = torch.zeros_like(inp["ckv_pool"])
+    ckv[..., 0] = 1.0
+    inp["ckv_pool"] = ckv
+    inp["w_uv"] = _bf16(np.broadcast_to(np.eye(64), (3, 64, 64)))
+    # keep the scores non-trivial through the rope part
+    dec, ab, _, _ = _run_both(inp)
+    assert np.abs(dec[..., 0] - 1.0).max() <= 1e-13
+    assert np.abs(dec[..., 1:]).max() == 0.0
+    assert np.abs(ab[..., 0] - 1.0).max() <= 1e-13
+
+
+def test_single_token_returns_its_value():
+    w = workload("dsv3", batch=3, heads=4, seq_len=1)
+    inp = make_inputs(w, seed=4)
+    dec, ab, _, lse = _run_both(inp)
+    for b, (c, _r) in enumerate(_dense_cache(inp)):
+        v = np.einsum("c,hce->he", c[0], _f64(inp["w_uv"]))
+        np.testing.assert_allclose(dec[b, 0], v, rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(ab[b, 0], v, rtol=1e-13, atol=1e-15)
+
+
+def test_zero_query_gives_mean_value():
+    w = SMALL["ragged"]
+    inp = make_inputs(w, seed=5)
+    inp["q_c"] = torch.zeros_like(inp["q_c"])
+    inp["q_r"] = torch.zeros_like(inp["q_r"])
+    dec, ab, _, lse = _run_both(inp)
+    for b, (c, _r) in enumerate(_dense_cache(inp)):
+        mean_v = np.einsum("c,hce->he", c.mean(axis=0), _f64(inp["w_uv"]))
+        np.testing.assert_allclose(dec[b, 0], mean_v, rtol=1e-12, atol=1e-14)
+        # lse of equal scores 0 over L tokens is log L
+        np.testing.assert_allclose(lse[b, 0], math.log(c.shape[0]), rtol=1e-13)
+
+
+def test_duplicated_tokens_leave_result_unchanged():
+    w = workload("dsv3", batch=1, heads=3, seq_len=96)
+    inp = make_inputs(w, seed=6)
+    dec, _, _, _ = _run_both(inp)
+    # same logical sequence with every token repeated twice
+    (c, r), = _dense_cache(inp)
+    c2, r2 = np.repeat(c, 2, axis=0), np.repeat(r, 2, axis=0)
+    L2, P = c2.shape[0], 64
+    n_pages = (L2 + P - 1) // P
+    pool_c = np.zeros((n_pages * P, c.shape[1]))
+    pool_r = np.zeros((n_pages * P, r.shape[1]))
+    pool_c[:L2], pool_r[:L2] = c2, r2
+    inp2 = dict(inp)
+    inp2["ckv_pool"] = _bf16(pool_c.reshape(n_pages, P, -1))
+    inp2["kr_pool"] = _bf16(pool_r.reshape(n_pages, P, -1))
+    inp2["block_table"] = torch.arange(n_pages, dtype=torch.int32)[None]
+    inp2["seq_lens"] = torch.tensor([L2], dtype=torch.int32)
+    dec2, _, _, _ = _run_both(inp2)
+    np.testing.assert_allclose(dec2, dec, rtol=1e-12, atol=1e-15)
+
+
+def test_common_score_shift_leaves_result_unchanged():
+    # append one rope dimension with q_r = alpha and k_R = 1 for every token:
+    # every score moves by scale*alpha, which softmax ignores (fixed scale).
+    w = workload("retrofit", batch=2, heads=3, seq_len=100)
+    inp = make_inputs(w, seed=7)
+    scale = oracle.default_scale(w.d_nope, w.d_rope)
+    dec, _, _, _ = _run_both(inp, scale=scale)
+    inp2 = dict(inp)
+    inp2["q_r"] = torch.cat([inp["q_r"], torch.full_like(inp["q_r"][..., :1], 3.0)], dim=-1)
+    inp2["kr_pool"] = torch.cat([inp["kr_pool"], torch.ones_like(inp["kr_pool"][..., :1])], dim=-1)
+    dec2, ab2, _, _ = _run_both(inp2, scale=scale)
+    np.testing.assert_allclose(dec2, dec, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(ab2, dec, rtol=1e-12, atol=1e-15)
+
+
+def test_two_token_closed_form_pins_scale():
+    # nope part silenced (q_c = 0); rope scores x and 0 => weights are logistic
+    # in scale*x with scale = 1/sqrt(192) for the DeepSeek dims.
+    w = workload("dsv3", batch=1, heads=2, seq_len=2)
+    inp = make_inputs(w, seed=8)
+    inp["q_c"] = torch.zeros_like(inp["q_c"])
+    qr = torch.zeros_like(inp["q_r"])
+    qr[..., 0] = 6.0
+    qr[0, 0, 1, 0] = -2.5
+    inp["q_r"] = qr
+    kr = torch.zeros_like(inp["kr_pool"])
+    page = int(inp["block_table"][0, 0])
+    kr[page, 0, 0] = 1.0
+    inp["kr_pool"] = kr
+    dec, ab, _, _ = _run_both(inp)
+    (c, _r), = _dense_cache(inp)
+    v = np.einsum("sc,hce->she", c, _f64(inp["w_uv"]))
+    tau = 1.0 / math.sqrt(192.0)
+    for h, x in ((0, 6.0), (1, -2.5)):
+        p0 = scipy.special.expit(tau * x)
+        expect = p0 * v[0, h] + (1 - p0) * v[1, h]
+        np.testing.assert_allclose(dec[0, 0, h], expect, rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(ab[0, 0, h], expect, rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("name", ["dsv3", "retrofit"])
+def test_rope_argmax_and_mask(name):
+    # W_UK = 0 silences the nope part. One visible token gets a rope score 60
+    # above all others => the output is its value. A token in the unused tail of
+    # the last page gets an even larger score but lies beyond L => ignored.
+    w = SMALL[name]
+    inp = make_inputs(w, seed=9, seq_lens=[w.seq_len - 5] * w.batch)
+    inp["w_uk"] = torch.zeros_like(inp["w_uk"])
+    scale = oracle.default_scale(w.d_nope, w.d_rope)
+    qr = torch.zeros_like(inp["q_r"])
+    qr[..., 0] = 60.0 / scale
+    inp["q_r"] = qr
+    kr = torch.zeros_like(inp["kr_pool"])
+    P = w.page_size
+    star = {}
+    for b in range(w.batch):
+        L = int(inp["seq_lens"][b])
+        t_star = (37 * (b + 1)) % (L - w.n_q + 1)          # visible to every query
+        pg = int(inp["block_table"][b, t_star // P])
+        kr[pg, t_star % P, 0] = 1.0
+        tail = L + 2                                         # beyond L, same last page
+        pg_t = int(inp["block_table"][b, tail // P])
+        kr[pg_t, tail % P, 0] = 2.0
+        star[b] = t_star
+    inp["kr_pool"] = kr
+    dec, ab, _, _ = _run_both(inp, scale=scale)
+    for b, (c, _r) in enumerate(_dense_cache(inp)):
+        v = np.einsum("c,hce->he", c[star[b]], _f64(inp["w_uv"]))
+        for i in range(w.n_q):
+            np.testing.assert_allclose(dec[b, i], v, rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(ab[b, i], v, rtol=1e-12, atol=1e-14)
+
+
+def test_causal_pair_equals_prefix_decode():
+    # query 0 of a two-query step sees exactly the prefix of length L-1
+    w = SMALL["retrofit"]
+    inp = make_inputs(w, seed=10)
+    dec, _, _, _ = _run_both(inp)
+    single = dict(inp)
+    single["q_c"] = inp["q_c"][:, :1].contiguous()
+    single["q_r"] = inp["q_r"][:, :1].contiguous()
+    single["seq_lens"] = inp["seq_lens"] - 1
+    dec0, _, _, _ = _run_both(single, scale=oracle.default_scale(w.d_nope, w.d_rope))
+    np.testing.assert_allclose(dec[:, 0], dec0[:, 0], rtol=1e-12, atol=1e-15)
+    # and query 1 sees the whole sequence
+    last = dict(inp)
+    last["q_c"] = inp["q_c"][:, 1:].contiguous()
+    last["q_r"] = inp["q_r"][:, 1:].contiguous()
+    dec1, _, _, _ = _run_both(last, scale=oracle.default_scale(w.d_nope, w.d_rope))
+    np.testing.assert_allclose(dec[:, 1], dec1[:, 0], rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# paging: gather bits and table invariance
+# ---------------------------------------------------------------------------
+
+def test_gather_is_bit_copy():
+    w = SMALL["ragged"]
+    inp = make_inputs(w, seed=11)
+    got = oracle.gather(inp["ckv_pool"], inp["block_table"], inp["seq_lens"], w.page_size)
+    bits = inp["ckv_pool"].view(torch.int16).numpy().view(np.uint16)
+    table, lens = inp["block_table"].numpy(), inp["seq_lens"].numpy()
+    for b, L in enumerate(lens):
+        t = np.arange(L)
+        np.testing.assert_array_equal(got[b, :L], bits[table[b, t // 64], t % 64])
+        assert not got[b, L:].any()
+
+
+def test_page_permutation_invariance_is_exact():
+    w = SMALL["dsv3"]
+    inp = make_inputs(w, seed=12)
+    dec, ab, o_lat, lse = _run_both(inp)
+    g = torch.Generator().manual_seed(99)
+    n = inp["ckv_pool"].shape[0]
+    perm = torch.randperm(n, generator=g)               # new physical slot of old page k
+    inp2 = dict(inp)
+    inp2["ckv_pool"] = torch.empty_like(inp["ckv_pool"])
+    inp2["kr_pool"] = torch.empty_like(inp["kr_pool"])
+    inp2["ckv_pool"][perm] = inp["ckv_pool"]
+    inp2["kr_pool"][perm] = inp["kr_pool"]
+    tbl = inp["block_table"].clone()
+    used = tbl >= 0
+    tbl[used] = perm[tbl[used].long()].to(torch.int32)
+    inp2["block_table"] = tbl
+    dec2, ab2, o_lat2, lse2 = _run_both(inp2)
+    np.testing.assert_array_equal(dec2, dec)
+    np.testing.assert_array_equal(ab2, ab)
+    np.testing.assert_array_equal(lse2, lse)
+
+
+def test_bad_tables_are_rejected():
+    w = SMALL["dsv3"]
+    inp = make_inputs(w, seed=13)
+    args = lambda d: [d[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table",
+                                     "seq_lens", "w_uk", "w_uv")]
+    bad = dict(inp)
+    bad["block_table"] = inp["block_table"].clone()
+    bad["block_table"][0, 1] = inp["ckv_pool"].shape[0]       # page id out of range
+    with pytest.raises(ValueError):
+        oracle.decode_decompress(*args(bad))
+    bad2 = dict(inp)
+    bad2["seq_lens"] = inp["seq_lens"].clone()
+    bad2["seq_lens"][1] = inp["block_table"].shape[1] * 64 + 1  # beyond the table
+    with pytest.raises(ValueError):
+        oracle.decode_decompress(*args(bad2))
+
+
+# ---------------------------------------------------------------------------
+# split windows and the log-sum-exp merge
+# ---------------------------------------------------------------------------
+
+def test_window_partials_combine_to_full_result():
+    w = SMALL["retrofit"]
+    inp = make_inputs(w, seed=14)
+    scale = oracle.default_scale(w.d_nope, w.d_rope)
+    q = torch.cat([inp["q_c"][..., :w.d_latent], inp["q_r"]], dim=-1)  # any bf16 query
+    common = (inp["ckv_pool"], inp["kr_pool"], inp["block_table"], inp["seq_lens"], scale)
+    o_full, lse_full = oracle.attend_latent(q, *common)
+    edges = [0, 17, 64, 64, 100, 500, 1000]      # includes an empty and a past-the-end window
+    parts = [oracle.attend_latent(q, *common, t_lo=a, t_hi=b) for a, b in zip(edges, edges[1:])]
+    o_part = np.stack([p[0] for p in parts], axis=-2).reshape(-1, len(parts), w.d_latent)
+    lse_part = np.stack([p[1] for p in parts], axis=-1).reshape(-1, len(parts))
+    assert np.isneginf(lse_part[:, 2]).all() and np.isneginf(lse_part[:, 5]).all()
+    o, lse = oracle.combine(o_part, lse_part)
+    np.testing.assert_allclose(o, o_full.reshape(-1, w.d_latent), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(lse, lse_full.ravel(), rtol=1e-13)
+
+
+def test_combine_textbook_cases():
+    rng = np.random.default_rng(0)
+    o_part = rng.standard_normal((3, 4, 5))
+    lse_part = np.array([[0.0, -np.inf, 1.0, 2.0],
+                         [-np.inf] * 4,
+                         [5.0, 5.0, 5.0, 5.0]])
+    o, lse = oracle.combine(o_part, lse_part)
+    w0 = scipy.special.softmax(np.array([0.0, 1.0, 2.0]))
+    np.testing.assert_allclose(o[0], w0 @ o_part[0, [0, 2, 3]], rtol=1e-14)
+    np.testing.assert_allclose(lse[0], scipy.special.logsumexp([0.0, 1.0, 2.0]), rtol=1e-15)
+    assert not o[1].any() and np.isneginf(lse[1])
+    np.testing.assert_allclose(o[2], o_part[2].mean(axis=0), rtol=1e-14)
+    np.testing.assert_allclose(lse[2], 5.0 + math.log(4.0), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# absorb-in / absorb-out: operand orientation and brute force
+# ---------------------------------------------------------------------------
+
+def _onehot_weights(H, rows, cols, rng):
+    """W[h][d][c] = 1 where c = perm_h(d) (rows <= cols)."""
+    W = np.zeros((H, rows, cols))
+    perms = [rng.permutation(cols)[:rows] for _ in range(H)]
+    for h in range(H):
+        W[h, np.arange(rows), perms[h]] = 1.0
+    return W, perms
+
+
+def test_absorb_q_orientation_and_brute_force():
+    rng = np.random.default_rng(1)
+    H, d_n, d_c, T = 3, 48, 64, 5
+    q = _bf16(rng.standard_normal((T, H, d_n)))
+    W, perms = _onehot_weights(H, d_n, d_c, rng)
+    got = oracle.absorb_q(q, _bf16(W))
+    qd = _f64(q)
+    for h in range(H):
+        expect = np.zeros((T, d_c))
+        expect[:, perms[h]] = qd[:, h]
+        np.testing.assert_array_equal(got[:, h], expect)
+    Wr = _bf16(rng.standard_normal((H, d_n, d_c)) / 8)
+    got = oracle.absorb_q(q, Wr)
+    np.testing.assert_allclose(got, np.einsum("thd,hdc->thc", qd, _f64(Wr)), rtol=1e-12,
+                               atol=1e-13)
+
+
+def test_absorb_out_orientation_and_brute_force():
+    rng = np.random.default_rng(2)
+    H, d_c, d_v, T = 3, 64, 128, 4
+    o = _bf16(rng.standard_normal((T, H, d_c)))
+    Wt, perms = _onehot_weights(H, d_c, d_v, rng)        # W[h][c][e] = 1 at e = perm_h(c)
+    got = oracle.absorb_out(o, _bf16(Wt))
+    od = _f64(o)
+    for h in range(H):
+        expect = np.zeros((T, d_v))
+        expect[:, perms[h]] = od[:, h]
+        np.testing.assert_array_equal(got[:, h], expect)
+    Wr = _bf16(rng.standard_normal((H, d_c, d_v)) / 8)
+    got = oracle.absorb_out(o, Wr)
+    np.testing.assert_allclose(got, np.einsum("thc,hce->the", od, _f64(Wr)), rtol=1e-12,
+                               atol=1e-13)
+    # fp64 input path agrees with the bf16 path on bf16-exact values
+    np.testing.assert_array_equal(oracle.absorb_out(od, Wr), got)
