@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark: MLA decode over a paged latent cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload long|dsv3|ragged|retrofit|tiny]
+
+A step is one pass of the whole decode path -- absorb-in, split-KV decode,
+log-sum-exp combine, absorb-out -- over one batch of the workload (default:
+batch 16, 128 heads, 65536 cached tokens per sequence, d_c 512, d_R 64,
+page_size 64, shuffled page table). Inputs (1.2 GB of latent cache) exceed the
+126 MB L2, so no flush is needed between steps. With N GPUs each rank runs its
+own replica (no collective on the data path; weak scaling) and the time is the
+maximum over ranks. One JSON line is printed by rank 0.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (each
+step a bounded sample of the same workload) and prints the same line with
+"impl": "reference".
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode KV-tokens/s per B200 (bf16) + % of HBM/tensor roofline vs CPU oracle"
+UNIT = "KV-tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# DRAM bytes per launch of the decode kernel from an ncu capture, keyed by the
+# sha256 of the kernel source it was taken on; reported only while the source
+# is unchanged.
+TRAFFIC = {}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    for f in ("decode.cuh", "common.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "mla_latent_kv_18_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _workload_desc(w, lens):
+    return (f"{w.name}: batch {w.batch}, n_q {w.n_q}, heads {w.heads}, d_nope {w.d_nope}, "
+            f"d_c {w.d_latent}, d_R {w.d_rope}, page {w.page_size}, "
+            f"seq {'U[%d,%d]' % w.ragged if w.ragged else w.seq_len}, "
+            f"{'identity' if w.table == 'identity' else 'shuffled'} page table")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons via NVML during the run (read only)."""
+
+    def __init__(self, index, period_s=0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((time.time(), mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        nv = self.nv
+        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-5:]
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        seen = set()
+        for s in win:
+            for k, bit in names.items():
+                if s[2] & bit and k != "gpu_idle":
+                    seen.add(k)
+        return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(seen), "samples": len(win)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(a):
+    """Times the fp64 CPU oracle on bounded samples of the workload."""
+    world, rank, _ = _dist_init()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    from mla_latent_kv_18_b200.inputs import make_inputs, workload
+    w = workload(a.workload)
+    inp = make_inputs(w, seed=0)
+    cores = oracle.num_threads()
+    R = w.n_q * w.heads
+    rng = np.random.default_rng(0)
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    lens = inp["seq_lens"].numpy()
+
+    def step():
+        sel = rng.choice(w.batch * R, size=cores, replace=False)
+        oracle.decode_absorbed(*args, sel=sel)
+        return float(sum(lens[s // R] for s in sel)) / R
+
+    for _ in range(a.warmup):
+        step()
+    t0 = time.perf_counter()
+    tokens = sum(step() for _ in range(a.steps))
+    dt = time.perf_counter() - t0
+    value = tokens / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * dt / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": _workload_desc(w, lens), "batch": w.batch,
+                       "seq_len": w.seq_len or list(w.ragged), "heads": w.heads,
+                       "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{cores} random (sequence, head) rows per step, each the "
+                                       "full absorbed fp64 oracle over the sequence's tokens"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(w, inp, target_s):
+    """Oracle (absorbed fp64 path, all host cores) on a bounded sample of rows."""
+    import numpy as np
+    import oracle
+    cores = oracle.num_threads()
+    R = w.n_q * w.heads
+    lens = inp["seq_lens"].numpy()
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    rng = np.random.default_rng(1)
+    n = cores
+    t0 = time.perf_counter()
+    sel = rng.choice(w.batch * R, size=n, replace=False)
+    oracle.decode_absorbed(*args, sel=sel)
+    dt = time.perf_counter() - t0
+    if dt < target_s / 2:
+        n = int(min(w.batch * R, max(n, n * target_s / max(dt, 1e-3))))
+        sel = rng.choice(w.batch * R, size=n, replace=False)
+        t0 = time.perf_counter()
+        oracle.decode_absorbed(*args, sel=sel)
+        dt = time.perf_counter() - t0
+    tokens = float(sum(lens[s // R] for s in sel)) / R
+    return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} random (sequence, head) rows of the workload, full absorbed fp64 "
+                      f"oracle over each row's tokens, {dt:.1f} s; KV-tokens counted as "
+                      "rows x tokens / rows-per-sequence"}
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        return run_reference(a)
+
+    import torch
+    import torch.distributed as dist
+    world, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from mla_latent_kv_18_b200 import build as mla_build
+    mla_build.build()
+    from mla_latent_kv_18_b200 import api
+    from mla_latent_kv_18_b200.inputs import make_inputs, to_device, workload
+
+    w = workload(a.workload)
+    inp = make_inputs(w, seed=rank)
+    d = to_device(inp, dev)
+    lens = inp["seq_lens"].numpy()
+    dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
+    T = api.tile_tokens(dims)
+    total_tiles = int(sum((int(L) + T - 1) // T for L in lens))
+    dec = api.Decoder(dims, w.batch, d["block_table"].shape[1], total_tiles, dev)
+    stream = torch.cuda.current_stream()
+    tokens_per_step = float(lens.sum())
+
+    def step(ev=None):
+        api.absorb_q(d["q_c"], d["q_r"], d["w_uk"], dims, out=dec.q)
+        if ev is not None:
+            ev[0].record(stream)
+        api.decode_splitkv(dec.q, d["ckv_pool"], d["kr_pool"], d["block_table"], d["seq_lens"],
+                           dims, dec.num_parts, workspace=dec.workspace)
+        if ev is not None:
+            ev[1].record(stream)
+        api.combine(dec.workspace, d["seq_lens"], dec.max_pages, dims, dec.num_parts,
+                    o_lat=dec.o_lat, lse_out=dec.lse)
+        api.absorb_out(dec.o_lat, d["w_uv"], dims, out=dec.out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(local).start()
+    for _ in range(max(3, a.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(a.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    ms = start.elapsed_time(end)
+    decode_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    assert api.get_device_error() == 0
+
+    # end to end through the same calls: per step, the step's inputs come from
+    # pinned host memory and the output goes back to pinned host memory.
+    h = {k: inp[k].pin_memory() for k in ("q_c", "q_r", "block_table", "seq_lens")}
+    h_out = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, a.steps // 2)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(e_steps):
+        for k, t in h.items():
+            d[k].copy_(t, non_blocking=True)
+        step()
+        h_out.copy_(dec.out, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = e_start.elapsed_time(e_end)
+    sampler.stop()
+
+    def allmax(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms, e_ms, decode_ms = allmax(ms), allmax(e_ms), allmax(decode_ms)
+    value = world * tokens_per_step * a.steps / (ms / 1e3)
+    e2e_value = world * tokens_per_step * e_steps / (e_ms / 1e3)
+
+    hbm, tflops, src = _peaks()
+    R = w.n_q * w.heads
+    kv_bytes = tokens_per_step * (w.d_latent + w.d_rope) * 2
+    q_bytes = w.batch * R * (w.d_latent + w.d_rope) * 2
+    alg_bytes = kv_bytes + q_bytes
+    vis = sum(sum(int(L) - w.n_q + i + 1 for i in range(w.n_q)) for L in lens)
+    alg_flops = vis * w.heads * (2 * (w.d_latent + w.d_rope) + 2 * w.d_latent)
+    achieved = alg_bytes / (decode_ms / 1e3) / 1e9
+    tr = TRAFFIC.get(_src_hash())
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": tr, "kernel": "decode_pair_kernel"
+            if w.d_latent == 512 else "decode_single_kernel",
+            "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+            "algorithmic_bytes_per_launch": alg_bytes,
+            "decode_ms_per_launch": decode_ms,
+            "tensor_achieved_tflops": alg_flops / (decode_ms / 1e3) / 1e12,
+            "tensor_peak_tflops": tflops,
+            "tensor_frac": alg_flops / (decode_ms / 1e3) / 1e12 / tflops}
+
+    clocks = sampler.summary(wall0, wall1)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": _workload_desc(w, lens), "batch": w.batch,
+                       "seq_len": w.seq_len or list(w.ragged), "heads": w.heads,
+                       "kv_tokens_per_step": tokens_per_step, "num_parts": dec.num_parts,
+                       "l2": "inputs larger than L2 (latent cache %.2f GB), no flush" % (kv_bytes / 1e9),
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "clocks": clocks,
+            "gpu_launches": 4 * a.steps}
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, a.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) library for DeepSeek-style
+ * Multi-head Latent Attention (MLA) decode over a paged latent KV cache,
+ * computed through matrix absorption.
+ *
+ * The method ("MLA operator design" page, bhfrc.com/news/60867, §1 and §4;
+ * "MHA2MLA" page, lpnh.cn/news/2494972, §2.1): per token and layer the cache
+ * keeps a d_c-wide latent c_KV plus a d_R-wide decoupled-RoPE key k_R. A decode
+ * step with query q = [q_c (d_n per head) | q_r (d_R per head)] computes, per
+ * head h,
+ *     out_h = softmax(scale * (q_c W_UK[h] c_KV^T + q_r k_R^T)) c_KV W_UV[h]
+ * in four calls:
+ *     mla_absorb_q        Q = [q_c W_UK[h] | q_r]                (fold into latent space)
+ *     mla_decode_splitkv  per partition of the cache: o = softmax(Q [c_KV|k_R]^T) c_KV, lse
+ *     mla_combine         log-sum-exp merge of the partitions -> o_lat
+ *     mla_absorb_out      out = o_lat W_UV[h]                    (up-project once)
+ * so the per-head K and V are never materialised.
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless a parameter says "host". The
+ *     caller owns every buffer; the library allocates no device memory.
+ *   - bf16 means IEEE bfloat16 stored as 16-bit words; fp32 is float.
+ *   - Tensors are dense row-major unless a stride is given. Shapes are written
+ *     outermost first, e.g. [T, H, d] has d contiguous.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise, except mla_get_device_error.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     returned as MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED; nothing is written
+ *     in that case. Data-dependent errors found by the kernels (a page id
+ *     outside the pool, a sequence length beyond its table row or below n_q, a
+ *     bounded wait that ran out) are recorded in a device error word and read
+ *     back with mla_get_device_error; the affected outputs are then undefined
+ *     but every kernel still terminates.
+ *   - Results are deterministic: repeated calls with the same inputs and the
+ *     same num_parts give bitwise-identical outputs, independent of which
+ *     physical pages hold the tokens.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, inconsistent dims */
+    MLA_ERR_UNSUPPORTED = 2,   /* dims outside the compiled specialisations, no sm_100 device */
+    MLA_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+    MLA_ERR_DEVICE_BOUNDS = 4, /* (device word) bad page id or sequence length */
+    MLA_ERR_TIMEOUT = 5        /* (device word) a bounded wait inside a kernel ran out */
+} mla_status;
+
+/* Problem dimensions. Supported specialisations:
+ *   d_latent 512, d_rope 64   (DeepSeek-V2/V3: "MLA operator design" §3 constants)
+ *   d_latent  64, d_rope  8   (retrofitted MLA: "MHA2MLA" §3.2 configuration)
+ * with page_size 64, d_nope <= 128 and a multiple of 8, d_v <= 256 and a
+ * multiple of 8, and n_q * num_heads <= 128 query rows per sequence. */
+typedef struct {
+    int32_t num_heads;     /* H */
+    int32_t n_q;           /* query tokens per sequence in this step (1, or 2 for a causal pair) */
+    int32_t d_nope;        /* d_n: per-head non-RoPE query width (128 or 120) */
+    int32_t d_latent;      /* d_c: latent width of c_KV */
+    int32_t d_rope;        /* d_R: width of the decoupled RoPE key k_R */
+    int32_t d_v;           /* per-head value width (128) */
+    int32_t page_size;     /* tokens per cache page; must be 64 ("MLA operator design" §3) */
+    float softmax_scale;   /* <= 0 selects 1/sqrt(d_nope + d_rope) ("MLA operator design" §4) */
+} mla_dims;
+
+/* One page pool: element (page p, token j, channel c) is at
+ * base[p * page_stride + j * token_stride + c] (strides in elements).
+ * base must be 16-byte aligned and both strides multiples of 8 elements
+ * (16 bytes), as the tensor-memory-access engine requires. The c_KV and k_R
+ * pools may be separate tensors or two views of one interleaved
+ * [pages, 64, d_c + d_R] tensor. */
+typedef struct {
+    const void *base;
+    int64_t page_stride;
+    int64_t token_stride;
+} mla_pool;
+
+/*
+ * Absorb-in ("MLA operator design" §4, path B: q_abs = q_c . w_uk per head).
+ *   q_out[t, h, 0:d_c]       = bf16( sum_d q_c[t, h, d] * w_uk[h, d, :] )   (fp32 accumulation)
+ *   q_out[t, h, d_c:d_c+d_R] = q_r[t, h, :]                                 (bit copy)
+ * q_c   [T, H, d_nope] bf16      q_r  [T, H, d_rope] bf16
+ * w_uk  [H, d_nope, d_latent] bf16 (the page's w_uk[nh, dhc, dc] layout)
+ * q_out [T, H, d_latent + d_rope] bf16; T = num_tokens >= 0 (0 is a no-op).
+ * All pointers 16-byte aligned.
+ */
+mla_status mla_absorb_q(const mla_dims *dims, const void *q_c, const void *q_r, const void *w_uk,
+                        void *q_out, int32_t num_tokens, void *stream);
+
+/* Number of cache partitions mla_decode_splitkv should use for a batch whose
+ * sequences hold total_tiles 64-token tiles in all (sum of ceil(L_b / 64)),
+ * on a device with num_sms multiprocessors. Host-only arithmetic; returns >= 1. */
+int32_t mla_decode_num_parts(const mla_dims *dims, int64_t total_tiles, int32_t num_sms);
+
+/* Bytes of device workspace mla_decode_splitkv / mla_combine need for `batch`
+ * sequences and `num_parts` partitions. Layout (R = n_q * num_heads,
+ * S = batch + num_parts slots):
+ *   offset 0:                 o_part [S, R, d_latent] fp32 (normalised partial outputs)
+ *   offset align256(S*R*d_c*4): lse_part [S, R] fp32 (natural-log log-sum-exp of
+ *                             the scaled scores of each partial; -inf if empty)
+ * Returns 0 for invalid dims. */
+size_t mla_decode_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t num_parts);
+
+/*
+ * Split-KV decode in latent space (the absorbed score and value steps).
+ * The flattened list of tiles of all sequences (N tiles of 64 tokens for
+ * d_latent 512, of 128 tokens for d_latent 64) is cut into P = min(num_parts, N)
+ * contiguous ranges, range p holding tiles [floor(p N / P), floor((p+1) N / P));
+ * each range is processed by one CTA pair (d_latent 512) or one CTA
+ * (d_latent 64). For every (sequence, range) overlap it writes one slot of the
+ * workspace, slots numbered sequence-major:
+ *   s[r, t]  = scale * (Q[b, r, 0:d_c] . c_KV[t] + Q[b, r, d_c:] . k_R[t])
+ *   o[r, :]  = sum_t softmax(s[r, :])_t c_KV[t]       over the range's visible tokens
+ *   lse[r]   = log sum_t exp(s[r, t])
+ * Row r = i * H + h of sequence b is query i (0 <= i < n_q) of head h; it sees
+ * tokens t <= seq_lens[b] - n_q + i (seq_lens counts the tokens already in the
+ * cache, the n_q current ones included).
+ * Token t of sequence b is read from page block_table[b * max_pages_per_seq + t / 64],
+ * row t % 64 ("MLA operator design" §3 page table); entries past
+ * ceil(seq_lens[b] / 64) are never read.
+ *
+ * q           [batch, n_q * H, d_latent + d_rope] bf16 (the q_out of mla_absorb_q)
+ * ckv, kr     page pools (host structs describing device memory), num_pages pages each
+ * block_table [batch, max_pages_per_seq] int32
+ * seq_lens    [batch] int32, n_q <= seq_lens[b] <= max_pages_per_seq * 64
+ * workspace   >= mla_decode_workspace_bytes(dims, batch, num_parts) bytes, 256-byte aligned
+ * batch = 0 is a no-op.
+ */
+mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_pool *ckv,
+                              const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                              int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                              int32_t num_parts, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * Log-sum-exp merge of the partial results written by mla_decode_splitkv with
+ * the same dims, seq_lens, batch and num_parts:
+ *   L = log sum_s exp(lse_s),   o_lat[b, r, :] = bf16( sum_s exp(lse_s - L) o_s[r, :] )
+ * A row with no visible token gives o_lat = 0 and lse = -inf.
+ * o_lat   [batch, n_q * H, d_latent] bf16 (= [batch, n_q, H, d_latent])
+ * lse_out [batch, n_q * H] fp32, may be NULL.
+ */
+mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t workspace_bytes,
+                       const int32_t *seq_lens, int32_t max_pages_per_seq, int32_t batch,
+                       int32_t num_parts, void *o_lat, float *lse_out, void *stream);
+
+/*
+ * Absorb-out ("MHA2MLA" §2.1: v = c_kv W_uv, applied once to the latent result).
+ *   out[t, h, :] = bf16( sum_c o_lat[t, h, c] * w_uv[h, c, :] )   (fp32 accumulation)
+ * o_lat [T, H, d_latent] bf16, w_uv [H, d_latent, d_v] bf16, out [T, H, d_v] bf16.
+ */
+mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w_uv, void *out,
+                          int32_t num_tokens, void *stream);
+
+/* Synchronises `stream`, returns in *code (host pointer) the first error a
+ * kernel of this library recorded on the current device since the last call
+ * (MLA_OK if none), and clears it. */
+mla_status mla_get_device_error(int32_t *code, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *mla_status_string(int32_t status);
+
+/*
+ * Host-side partition plan, the same arithmetic the kernels use. For
+ * seq_lens_host[batch] (host array) and num_parts, fills (host arrays, any may
+ * be NULL):
+ *   part_first[b]  first partition that covers sequence b (-1 if it has no tile)
+ *   slot_count[b]  number of partial slots of sequence b
+ *   slot_base[b]   index of its first slot in the workspace
+ * and returns the total number of slots used (<= batch + num_parts), or -1 on
+ * invalid arguments.
+ */
+int64_t mla_decode_plan(const mla_dims *dims, const int32_t *seq_lens_host,
+                        int32_t max_pages_per_seq, int32_t batch, int32_t num_parts,
+                        int32_t *part_first, int32_t *slot_count, int64_t *slot_base);
+
+/*
+ * Test hook for the bounded waits: launches one block that waits on a barrier
+ * nothing will complete, with a limit of timeout_ns nanoseconds, after which it
+ * records MLA_ERR_TIMEOUT in the device error word and returns. Lets a test
+ * check that a wait which runs out ends the kernel cleanly with a readable
+ * status.
+ */
+mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

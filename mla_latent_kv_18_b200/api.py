@@ -1,0 +1,202 @@
+"""Python API over the C ABI: MLA decode with matrix absorption on a paged
+latent cache. PyTorch supplies device memory and the current stream only;
+every step runs in the library's sm_100a kernels.
+
+    q   = absorb_q(q_c, q_r, w_uk)                         # [B, n_q, H, d_c + d_R]
+    ws, parts = decode_splitkv(q, ckv_pool, kr_pool, block_table, seq_lens)
+    o, lse = combine(ws, seq_lens, parts, ...)             # [B, n_q, H, d_c]
+    out = absorb_out(o, w_uv)                              # [B, n_q, H, d_v]
+
+or ``decode(...)`` for all four.
+"""
+import ctypes
+
+import torch
+
+from . import _binding as _b
+
+_NUM_SMS = {}
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _num_sms(device):
+    idx = torch.device(device).index
+    if idx is None:
+        idx = torch.cuda.current_device()
+    if idx not in _NUM_SMS:
+        _NUM_SMS[idx] = torch.cuda.get_device_properties(idx).multi_processor_count
+    return _NUM_SMS[idx]
+
+
+def make_dims(heads, n_q, d_nope, d_latent, d_rope, d_v, page_size=64, scale=0.0):
+    return _b.MLADims(heads, n_q, d_nope, d_latent, d_rope, d_v, page_size, float(scale))
+
+
+def dims_for(q_c, q_r, w_uk, w_uv, page_size=64, scale=0.0):
+    """Dims from tensor shapes: q_c [B, n_q, H, d_n], q_r [.., d_R], w_uk [H, d_n, d_c],
+    w_uv [H, d_c, d_v]."""
+    H, d_n, d_c = w_uk.shape
+    return make_dims(H, q_c.shape[1], d_n, d_c, q_r.shape[-1], w_uv.shape[-1], page_size, scale)
+
+
+def _pool(t):
+    """A [pages, 64, C] (possibly channel-sliced) bf16 view -> mla_pool."""
+    assert t.dtype == torch.bfloat16 and t.dim() == 3 and t.stride(2) == 1
+    return _b.MLAPool(t.data_ptr(), t.stride(0), t.stride(1))
+
+
+def absorb_q(q_c, q_r, w_uk, dims, out=None, stream=None):
+    T = q_c.numel() // (dims.num_heads * dims.d_nope)
+    if out is None:
+        out = torch.empty(q_c.shape[:-1] + (dims.d_latent + dims.d_rope,), dtype=torch.bfloat16,
+                          device=q_c.device)
+    _b.check(_b.lib.mla_absorb_q(ctypes.byref(dims), _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(out),
+                                 T, _stream(stream)), "mla_absorb_q")
+    return out
+
+
+def num_parts_for(dims, total_tiles, device=None):
+    return _b.lib.mla_decode_num_parts(ctypes.byref(dims), int(total_tiles),
+                                       _num_sms(device or torch.cuda.current_device()))
+
+
+def tile_tokens(dims):
+    return 64 if dims.d_latent == 512 else 128
+
+
+def workspace_bytes(dims, batch, num_parts):
+    return _b.lib.mla_decode_workspace_bytes(ctypes.byref(dims), batch, num_parts)
+
+
+def alloc_workspace(dims, batch, num_parts, device):
+    nbytes = workspace_bytes(dims, batch, num_parts)
+    if nbytes == 0:
+        raise _b.MLAError(1, "mla_decode_workspace_bytes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def workspace_views(ws, dims, batch, num_parts):
+    """(o_part [slots, R, d_c] fp32, lse_part [slots, R] fp32) views of a workspace."""
+    slots = batch + num_parts
+    R = dims.n_q * dims.num_heads
+    o_bytes = (slots * R * dims.d_latent * 4 + 255) // 256 * 256
+    o = ws[:slots * R * dims.d_latent * 4].view(torch.float32).view(slots, R, dims.d_latent)
+    lse = ws[o_bytes:o_bytes + slots * R * 4].view(torch.float32).view(slots, R)
+    return o, lse
+
+
+def plan(dims, seq_lens_host, max_pages, num_parts):
+    """Host replica of the kernels' partition plan: (part_first, slot_count, slot_base, slots)."""
+    lens = torch.as_tensor(seq_lens_host, dtype=torch.int32).contiguous()
+    B = lens.numel()
+    pf = torch.empty(B, dtype=torch.int32)
+    cnt = torch.empty(B, dtype=torch.int32)
+    base = torch.empty(B, dtype=torch.int64)
+    total = _b.lib.mla_decode_plan(ctypes.byref(dims), _ptr(lens), max_pages, B, num_parts,
+                                   _ptr(pf), _ptr(cnt), _ptr(base))
+    if total < 0:
+        raise _b.MLAError(1, "mla_decode_plan")
+    return pf, cnt, base, total
+
+
+def decode_splitkv(q, ckv_pool, kr_pool, block_table, seq_lens, dims, num_parts,
+                   workspace=None, stream=None):
+    B = block_table.shape[0]
+    if workspace is None:
+        workspace = alloc_workspace(dims, B, num_parts, q.device)
+    ckv, kr = _pool(ckv_pool), _pool(kr_pool)
+    _b.check(_b.lib.mla_decode_splitkv(ctypes.byref(dims), _ptr(q), ctypes.byref(ckv),
+                                       ctypes.byref(kr), ckv_pool.shape[0], _ptr(block_table),
+                                       block_table.shape[1], _ptr(seq_lens), B, num_parts,
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+             "mla_decode_splitkv")
+    return workspace
+
+
+def combine(workspace, seq_lens, max_pages, dims, num_parts, o_lat=None, lse_out=None,
+            with_lse=True, stream=None):
+    B = seq_lens.shape[0]
+    R = dims.n_q * dims.num_heads
+    dev = workspace.device
+    if o_lat is None:
+        o_lat = torch.empty(B, dims.n_q, dims.num_heads, dims.d_latent, dtype=torch.bfloat16,
+                            device=dev)
+    if with_lse and lse_out is None:
+        lse_out = torch.empty(B, dims.n_q, dims.num_heads, dtype=torch.float32, device=dev)
+    _b.check(_b.lib.mla_combine(ctypes.byref(dims), _ptr(workspace), workspace.numel(),
+                                _ptr(seq_lens), max_pages, B, num_parts, _ptr(o_lat),
+                                _ptr(lse_out) if with_lse else None, _stream(stream)),
+             "mla_combine")
+    return o_lat, lse_out
+
+
+def absorb_out(o_lat, w_uv, dims, out=None, stream=None):
+    T = o_lat.numel() // (dims.num_heads * dims.d_latent)
+    if out is None:
+        out = torch.empty(o_lat.shape[:-1] + (dims.d_v,), dtype=torch.bfloat16, device=o_lat.device)
+    _b.check(_b.lib.mla_absorb_out(ctypes.byref(dims), _ptr(o_lat), _ptr(w_uv), _ptr(out), T,
+                                   _stream(stream)), "mla_absorb_out")
+    return out
+
+
+def get_device_error(stream=None):
+    code = ctypes.c_int32(0)
+    _b.check(_b.lib.mla_get_device_error(ctypes.byref(code), _stream(stream)),
+             "mla_get_device_error")
+    return code.value
+
+
+def debug_wait_timeout(timeout_ns, stream=None):
+    _b.check(_b.lib.mla_debug_wait_timeout(int(timeout_ns), _stream(stream)),
+             "mla_debug_wait_timeout")
+
+
+class Decoder:
+    """All four steps with fixed shapes; buffers allocated once (by PyTorch).
+
+    total_tiles: sum over sequences of ceil(L_b / tile_tokens) -- decides the
+    number of partitions; pass the host-side value when known.
+    """
+
+    def __init__(self, dims, batch, max_pages, total_tiles, device):
+        self.dims = dims
+        self.batch = batch
+        self.max_pages = max_pages
+        self.num_parts = num_parts_for(dims, total_tiles, device)
+        self.workspace = alloc_workspace(dims, batch, self.num_parts, device)
+        H, n_q = dims.num_heads, dims.n_q
+        self.q = torch.empty(batch, n_q, H, dims.d_latent + dims.d_rope, dtype=torch.bfloat16,
+                             device=device)
+        self.o_lat = torch.empty(batch, n_q, H, dims.d_latent, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(batch, n_q, H, dtype=torch.float32, device=device)
+        self.out = torch.empty(batch, n_q, H, dims.d_v, dtype=torch.bfloat16, device=device)
+
+    def __call__(self, q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv,
+                 stream=None):
+        absorb_q(q_c, q_r, w_uk, self.dims, out=self.q, stream=stream)
+        decode_splitkv(self.q, ckv_pool, kr_pool, block_table, seq_lens, self.dims, self.num_parts,
+                       workspace=self.workspace, stream=stream)
+        combine(self.workspace, seq_lens, self.max_pages, self.dims, self.num_parts,
+                o_lat=self.o_lat, lse_out=self.lse, stream=stream)
+        absorb_out(self.o_lat, w_uv, self.dims, out=self.out, stream=stream)
+        return self.out
+
+
+def decode(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, total_tiles=None,
+           scale=0.0, stream=None):
+    """One decode step. Returns (out [B,n_q,H,d_v], o_lat [B,n_q,H,d_c], lse [B,n_q,H])."""
+    dims = dims_for(q_c, q_r, w_uk, w_uv, ckv_pool.shape[1], scale)
+    if total_tiles is None:
+        T = tile_tokens(dims)
+        total_tiles = int(((seq_lens.to(torch.int64) + T - 1) // T).sum().item())
+    dec = Decoder(dims, block_table.shape[0], block_table.shape[1], total_tiles, q_c.device)
+    out = dec(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, stream=stream)
+    return out, dec.o_lat, dec.lse

@@ -1,0 +1,148 @@
+// Shared device/host helpers of the CUDA path: status codes, the device error
+// word, bounded mbarrier waits and the partition plan arithmetic.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace mla {
+
+// Mirrors mla_status in include/mla_decode.h.
+enum : int32_t {
+    kOk = 0,
+    kErrInvalidArg = 1,
+    kErrUnsupported = 2,
+    kErrCuda = 3,
+    kErrDeviceBounds = 4,
+    kErrTimeout = 5,
+};
+
+// First error recorded by any kernel of the library on this device.
+__device__ int32_t g_device_error;
+
+__device__ __forceinline__ void record_error(int32_t code) {
+    atomicCAS(&g_device_error, 0, code);
+}
+
+// Bounded wait on phase `parity` of the barrier at shared address `bar`.
+// Polls the CTA's abort flag and the global timer; after `timeout_ns` it
+// records kErrTimeout, raises the abort flag and returns false.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int32_t *abort_flag, int64_t timeout_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (static_cast<int64_t>(ptx::globaltimer_ns() - t0) > timeout_ns) {
+                record_error(kErrTimeout);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Partition plan. The tiles (tile_tokens tokens each) of all sequences are
+// laid end to end; partition p of P owns tiles [start(p), start(p+1)) with
+// start(p) = floor(p * N / P). A sequence b with n_b tiles starting at tile
+// offset O_b is covered by partitions part(O_b) .. part(O_b + n_b - 1) and
+// gets one partial slot per covering partition; slots are numbered
+// sequence-major.
+// ---------------------------------------------------------------------------
+
+__host__ __device__ __forceinline__ int64_t part_start(int64_t p, int64_t N, int64_t P) {
+    return (p * N) / P;
+}
+
+// Partition that owns tile t (0 <= t < N): the largest p with start(p) <= t.
+__host__ __device__ __forceinline__ int64_t part_of_tile(int64_t t, int64_t N, int64_t P) {
+    return ((t + 1) * P + N - 1) / N - 1;
+}
+
+// Usable length of sequence b and its tile count. Lengths outside
+// [n_q, max_pages * 64] are reported through `bad` and clamped.
+__host__ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_pages, int32_t n_q,
+                                                      bool *bad) {
+    const int64_t cap = static_cast<int64_t>(max_pages) * 64;
+    if (L < n_q || static_cast<int64_t>(L) > cap) *bad = true;
+    if (L < 0) L = 0;
+    if (static_cast<int64_t>(L) > cap) L = static_cast<int32_t>(cap);
+    return L;
+}
+
+__host__ __device__ __forceinline__ int64_t tiles_of_len(int32_t L, int32_t tile_tokens) {
+    return (static_cast<int64_t>(L) + tile_tokens - 1) / tile_tokens;
+}
+
+struct SeqCursor {
+    int32_t b;          // sequence index
+    int64_t tile_off;   // O_b
+    int64_t slot_base;  // S_b
+    int64_t total;      // N
+    int64_t parts;      // partitions in use: min(num_parts, N), so each owns >= 1 tile
+};
+
+__host__ __device__ __forceinline__ int64_t parts_in_use(int64_t num_parts, int64_t N) {
+    return N < num_parts ? N : num_parts;
+}
+
+// Warp-cooperative scan: the sequence whose tile range contains tile `ts`
+// (or the first sequence with a tile at or after ts), with its tile offset and
+// slot base. All 32 lanes must call it; every lane gets the result.
+__device__ inline SeqCursor find_sequence(const int32_t *seq_lens, int32_t batch, int32_t max_pages,
+                                          int32_t n_q, int32_t tile_tokens, int64_t P,
+                                          int64_t ts) {
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    int64_t N = 0;
+    for (int32_t base = 0; base < batch; base += 32) {
+        int32_t b = base + lane;
+        int64_t n = 0;
+        if (b < batch) n = tiles_of_len(clamp_len(seq_lens[b], max_pages, n_q, &bad), tile_tokens);
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        N += n;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(kErrDeviceBounds);
+    SeqCursor cur{batch, N, 0, N, parts_in_use(P, N)};
+    if (N == 0) return cur;
+    P = cur.parts;
+    int64_t O = 0, S = 0;
+    for (int32_t base = 0; base < batch; base += 32) {
+        int32_t b = base + lane;
+        int64_t n = 0;
+        if (b < batch) n = tiles_of_len(clamp_len(seq_lens[b], max_pages, n_q, &bad), tile_tokens);
+        // exclusive prefix of n across the warp
+        int64_t incl = n;
+        for (int o = 1; o < 32; o <<= 1) {
+            int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int64_t Ob = O + incl - n;
+        int64_t ns = 0;
+        if (n > 0) ns = part_of_tile(Ob + n - 1, N, P) - part_of_tile(Ob, N, P) + 1;
+        int64_t sincl = ns;
+        for (int o = 1; o < 32; o <<= 1) {
+            int64_t v = __shfl_up_sync(0xffffffffu, sincl, o);
+            if (lane >= o) sincl += v;
+        }
+        const int64_t Sb = S + sincl - ns;
+        const bool hit = (n > 0) && (Ob + n > ts);
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            cur.b = __shfl_sync(0xffffffffu, b, src);
+            cur.tile_off = __shfl_sync(0xffffffffu, Ob, src);
+            cur.slot_base = __shfl_sync(0xffffffffu, Sb, src);
+            return cur;
+        }
+        O += __shfl_sync(0xffffffffu, incl, 31);
+        S += __shfl_sync(0xffffffffu, sincl, 31);
+    }
+    return cur;
+}
+
+}  // namespace mla

@@ -1,0 +1,952 @@
+// Split-KV MLA decode in latent space on sm_100a tensor cores.
+//
+// What one partition computes (absorbed score and value steps; "MLA operator
+// design" page §4 path B, "MHA2MLA" page §2.1):
+//   S = Q [c_KV | k_R]^T                      (all heads share one latent KV)
+//   online softmax over the partition's tokens (fp32, exp2 domain)
+//   O = P c_KV                                (value product stays in latent space)
+//   partial = O / l,  lse = m * scale + ln l
+//
+// Two kernels share the pipeline shape: warp 0 streams KV pages with TMA into
+// a two-stage shared-memory ring, one thread of warp 1 issues tcgen05 MMAs
+// into tensor memory, and warps 2..5 run the softmax, rescale O when the
+// running maximum grows by more than 2^8, write P, and write the partials.
+//
+//  * decode_pair_kernel (d_c 512, d_R 64, page = tile = 64 tokens): a CTA pair
+//    on two SMs. The fp32 accumulator O[128 rows x 512] is exactly one SM's
+//    256 KB of tensor memory, so the pair splits it: cta_group::2 MMAs with
+//    M = 128 give each SM the O rows of its 64 query rows. QK^T splits the
+//    tile's 64 tokens (32 per SM); P.V splits the 512 latent columns (256 per
+//    SM, as two N = 256 MMAs). No MMA work is duplicated.
+//  * decode_single_kernel (d_c 64, d_R 8, tile = 128 tokens = 2 pages): one
+//    CTA, cta_group::1, M = 128 rows; the 8-wide RoPE key is padded to the
+//    16-wide MMA K step with a zero core-matrix column in shared memory.
+//
+// Every wait is bounded (see wait_bounded); data errors set the device error
+// word. The kernels never read block-table entries past a sequence's last
+// page.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+struct DecodeArgs {
+    const __nv_bfloat16 *q;      // [B, R, D]
+    const int32_t *block_table;  // [B, max_pages]
+    const int32_t *seq_lens;     // [B]
+    float *o_part;               // [slots, R, d_c]
+    float *lse_part;             // [slots, R]
+    int64_t timeout_ns;
+    int32_t max_pages;
+    int32_t batch;
+    int32_t num_pages;
+    int32_t num_parts;
+    int32_t n_q;
+    int32_t heads;
+    int32_t rows;                // R = n_q * heads (<= 128)
+    float scale;                 // softmax scale
+    float scale_log2;            // scale * log2(e)
+};
+
+constexpr int kDecodeThreads = 192;          // 6 warps
+constexpr int kSoftmaxWarp0 = 2;             // warps 2..5
+constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when max grows > 2^8
+
+// ------------------------------------------------------------------ helpers
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_global_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
+// 128-byte-swizzled K-major block whose rows are 128 bytes apart.
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// Iterates the (sequence, tile range) segments of one partition. Every thread
+// that walks it gets the same sequence of segments.
+struct SegmentWalker {
+    const int32_t *seq_lens;
+    int32_t batch, max_pages, n_q, tile_tokens;
+    int64_t N, P, p, te;
+    // current state
+    int32_t b;
+    int64_t O, S, tile;
+    // current segment
+    int32_t seg_b, L;
+    int64_t t_begin, t_end, slot;
+
+    __device__ bool next() {
+        while (tile < te && b < batch) {
+            bool bad = false;
+            const int32_t Lb = clamp_len(seq_lens[b], max_pages, n_q, &bad);
+            const int64_t n = tiles_of_len(Lb, tile_tokens);
+            if (n == 0) { ++b; continue; }
+            const int64_t pf = part_of_tile(O, N, P);
+            seg_b = b;
+            L = Lb;
+            t_begin = tile - O;
+            t_end = (te - O < n) ? (te - O) : n;
+            slot = S + (p - pf);
+            tile = O + t_end;
+            const int64_t pl = part_of_tile(O + n - 1, N, P);
+            S += pl - pf + 1;
+            O += n;
+            ++b;
+            return true;
+        }
+        return false;
+    }
+};
+
+// ===========================================================================
+// CTA-pair kernel: d_c = 512, d_R = 64
+// ===========================================================================
+namespace pair {
+constexpr int DC = 512, DR = 64, D = DC + DR;
+constexpr int NB = D / 64;                    // 9 K-blocks of 64 channels
+constexpr int ROWS_CTA = 64;                  // query rows per SM
+constexpr int TOK = 64;                       // tokens per tile (one page)
+constexpr int OWN = 32;                       // tokens per SM in QK^T
+constexpr uint32_t Q_BYTES = NB * ROWS_CTA * 128;           // 73728
+constexpr uint32_t STAGE_QK = NB * OWN * 128;               // 36864
+constexpr uint32_t STAGE_PV = 4 * TOK * 128;                // 32768 (4 channel blocks x 64 tokens)
+constexpr uint32_t STAGE_BYTES = STAGE_QK + STAGE_PV;       // 69632
+constexpr int STAGES = 2;
+constexpr uint32_t P_BYTES = ROWS_CTA * 128;                // 64 rows x 64 tokens bf16
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_STAGE = OFF_Q + Q_BYTES;
+constexpr uint32_t OFF_P = OFF_STAGE + STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 229376
+constexpr uint32_t MISC_BYTES = 2048;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr uint32_t TX_PER_CTA = STAGE_BYTES;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
+constexpr uint32_t TMEM_S = 256;               // two 32-column score buffers
+constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, 256, 0, 1);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert((OFF_STAGE % 1024) == 0 && (OFF_P % 1024) == 0 && (OFF_MISC % 1024) == 0, "align");
+}  // namespace pair
+
+// misc-region layout (both kernels)
+struct Misc {
+    uint64_t full[2], empty[2], s_full[2], s_free[2], p_ready[2], pv_done[2], q_ready, o_free;
+    uint64_t xbar[2], xlbar, drain;   // row-statistics exchange among softmax warps; MMA drain
+    uint32_t tmem_base;
+    int32_t abort_flag;
+    int32_t cur_b;
+    int32_t pad0;
+    int64_t cur_O, cur_S, cur_N;
+    float xmax[2][128];
+    float xl[128];
+};
+static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
+    decode_pair_kernel(const __grid_constant__ CUtensorMap map_ckv32,
+                       const __grid_constant__ CUtensorMap map_ckv64,
+                       const __grid_constant__ CUtensorMap map_kr32, const DecodeArgs args) {
+    using namespace pair;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_base);
+    Misc *misc = reinterpret_cast<Misc *>(smem + OFF_MISC);
+    volatile int32_t *abort_flag = &misc->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();      // 0 = leader
+    const int64_t part = blockIdx.x >> 1;
+    const int64_t P = args.num_parts;
+
+    auto bar = [&](const uint64_t *b) { return ptx::smem_u32(b); };
+    // address of a barrier of the leader CTA, as seen from this CTA
+    auto leader_bar = [&](const uint64_t *b) { return ptx::mapa(ptx::smem_u32(b), 0); };
+
+    // ---------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(bar(&misc->full[i]), 1);
+            ptx::mbar_init(bar(&misc->empty[i]), 1);
+            ptx::mbar_init(bar(&misc->s_full[i]), 1);
+            ptx::mbar_init(bar(&misc->s_free[i]), 8);
+            ptx::mbar_init(bar(&misc->p_ready[i]), 8);
+            ptx::mbar_init(bar(&misc->pv_done[i]), 1);
+        }
+        ptx::mbar_init(bar(&misc->q_ready), 8);
+        ptx::mbar_init(bar(&misc->o_free), 8);
+        ptx::mbar_init(bar(&misc->xbar[0]), 4);
+        ptx::mbar_init(bar(&misc->xbar[1]), 4);
+        ptx::mbar_init(bar(&misc->xlbar), 4);
+        ptx::mbar_init(bar(&misc->drain), 1);
+        misc->abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
+                                          P, 0);
+        const int64_t N = c.total;
+        const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
+        const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
+                                          P, ts);
+        if (lane == 0) {
+            misc->cur_b = s.b;
+            misc->cur_O = s.tile_off;
+            misc->cur_S = s.slot_base;
+            misc->cur_N = N;
+            ptx::prefetch_tensormap(&map_ckv32);
+            ptx::prefetch_tensormap(&map_ckv64);
+            ptx::prefetch_tensormap(&map_kr32);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<2>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
+        ptx::tmem_relinquish<2>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    SegmentWalker walk;
+    walk.seq_lens = args.seq_lens;
+    walk.batch = args.batch;
+    walk.max_pages = args.max_pages;
+    walk.n_q = args.n_q;
+    walk.tile_tokens = TOK;
+    walk.N = misc->cur_N;
+    walk.P = parts_in_use(P, walk.N);
+    walk.p = part;
+    walk.b = misc->cur_b;
+    walk.O = misc->cur_O;
+    walk.S = misc->cur_S;
+    if (part < walk.P) {
+        walk.tile = part_start(part, walk.N, walk.P);
+        walk.te = part_start(part + 1, walk.N, walk.P);
+    } else {
+        walk.tile = walk.te = 0;   // idle partition
+    }
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (ptx::elect_one()) {
+            const uint32_t full0 = (rank == 0) ? bar(&misc->full[0]) : leader_bar(&misc->full[0]);
+            const uint32_t full1 = (rank == 0) ? bar(&misc->full[1]) : leader_bar(&misc->full[1]);
+            int64_t k = 0;
+            bool bad_page = false;
+            while (!*abort_flag && walk.next()) {
+                const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
+                for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
+                    const int s = static_cast<int>(k & 1);
+                    int32_t page = trow[t];
+                    if (page < 0 || page >= args.num_pages) { bad_page = true; page = 0; }
+                    if (t + 2 < walk.t_end) {  // warm L2 two tiles ahead (own rows)
+                        int32_t pg2 = trow[t + 2];
+                        if (pg2 >= 0 && pg2 < args.num_pages) {
+                            for (int j = 0; j < 8; ++j)
+                                ptx::tma_prefetch_3d(&map_ckv32, 64 * j, OWN * rank, pg2);
+                            ptx::tma_prefetch_3d(&map_kr32, 0, OWN * rank, pg2);
+                        }
+                    }
+                    if (k >= 2 && !wait_bounded(bar(&misc->empty[s]), ((k >> 1) - 1) & 1,
+                                                abort_flag, args.timeout_ns))
+                        break;
+                    const uint32_t fb = s ? full1 : full0;
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(&misc->full[s]), 2 * TX_PER_CTA);
+                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    for (int j = 0; j < 8; ++j)
+                        ptx::tma_load_3d_pair(st + j * (OWN * 128), &map_ckv32, fb, 64 * j,
+                                              OWN * rank, page);
+                    ptx::tma_load_3d_pair(st + 8 * (OWN * 128), &map_kr32, fb, 0, OWN * rank, page);
+                    for (int u = 0; u < 4; ++u) {
+                        const int blk = 4 * (u >> 1) + 2 * static_cast<int>(rank) + (u & 1);
+                        ptx::tma_load_3d_pair(st + STAGE_QK + u * (TOK * 128), &map_ckv64, fb,
+                                              64 * blk, 0, page);
+                    }
+                }
+            }
+            if (bad_page) record_error(kErrDeviceBounds);
+            // drain: the leader waits until every issued stage has landed
+            if (rank == 0) {
+                for (int64_t kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk)
+                    wait_bounded(bar(&misc->full[kk & 1]), (kk >> 1) & 1, abort_flag,
+                                 args.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer (leader)
+        if (rank == 0 && ptx::elect_one()) {
+            int64_t k = 0;
+            int64_t g = 0;
+            bool ok = true;
+            auto issue_pv = [&](int64_t kp, bool first_of_seg) -> bool {
+                const int s = static_cast<int>(kp & 1);
+                if (!wait_bounded(bar(&misc->p_ready[s]), (kp >> 1) & 1, abort_flag, args.timeout_ns))
+                    return false;
+                ptx::tc_fence_after();
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES + STAGE_QK;
+                const uint32_t pbuf = base + OFF_P + s * P_BYTES;
+                for (int c = 0; c < 2; ++c) {
+                    for (int kk = 0; kk < TOK / 16; ++kk) {
+                        const uint64_t a = ptx::smem_desc(pbuf + kk * 32, 16, 1024, ptx::kSwizzle128B);
+                        const uint64_t b = ptx::smem_desc(st + (2 * c) * (TOK * 128) + kk * 2048,
+                                                          TOK * 128, 1024, ptx::kSwizzle128B);
+                        ptx::mma_bf16_ss<2>(tmem + TMEM_O + 128 * c, a, b, IDESC_PV,
+                                            (first_of_seg && kk == 0) ? 0u : 1u);
+                    }
+                }
+                ptx::mma_commit_pair(bar(&misc->empty[s]), 0x3);
+                ptx::mma_commit_pair(bar(&misc->pv_done[s]), 0x3);
+                return true;
+            };
+            while (ok && !*abort_flag && walk.next()) {
+                const int64_t k0 = k;
+                if (!wait_bounded(bar(&misc->q_ready), g & 1, abort_flag, args.timeout_ns)) break;
+                for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
+                    const int s = static_cast<int>(k & 1);
+                    if (!wait_bounded(bar(&misc->full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (k >= 2 && !wait_bounded(bar(&misc->s_free[s]), ((k >> 1) - 1) & 1,
+                                                abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    for (int j = 0; j < NB; ++j) {
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t a = ptx::smem_desc(base + OFF_Q + j * (ROWS_CTA * 128) + kk * 32,
+                                                              16, 1024, ptx::kSwizzle128B);
+                            const uint64_t b = ptx::smem_desc(st + j * (OWN * 128) + kk * 32, 16, 1024,
+                                                              ptx::kSwizzle128B);
+                            ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s, a, b, IDESC_QK,
+                                                (j | kk) ? 1u : 0u);
+                        }
+                    }
+                    ptx::mma_commit_pair(bar(&misc->s_full[s]), 0x3);
+                    if (k > k0) {
+                        if (k - 1 == k0 && g > 0) {
+                            if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag,
+                                              args.timeout_ns)) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!issue_pv(k - 1, k - 1 == k0)) { ok = false; break; }
+                    }
+                }
+                if (!ok) break;
+                // value product of the segment's last tile
+                if (k - 1 == k0 && g > 0) {
+                    if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag, args.timeout_ns))
+                        break;
+                }
+                if (!issue_pv(k - 1, k - 1 == k0)) break;
+                ++g;
+            }
+            // every MMA issued so far has finished before tensor memory is freed
+            ptx::mma_commit_pair(bar(&misc->drain), 0x1);
+            wait_bounded(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------ softmax / epilogue
+        const int q4 = warp & 3;                       // TMEM lane quadrant
+        const int lt = q4 * 32 + lane;                 // TMEM lane 0..127
+        const int row = lt & 63;                       // local query row
+        const int half = lt >> 6;                      // which 32 tokens of the tile
+        const int grow = ROWS_CTA * static_cast<int>(rank) + row;  // row within the sequence
+        const bool real_row = grow < args.rows;
+        const int qi = real_row ? grow / args.heads : 0;
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const int st_tid = threadIdx.x - kSoftmaxWarp0 * 32;   // 0..127
+        auto arrive_leader = [&](uint64_t *b) {
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) ptx::mbar_arrive(bar(b));
+                else ptx::mbar_arrive_cluster(leader_bar(b));
+            }
+        };
+        auto load_q = [&](int32_t b) {
+            const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
+            for (int idx = st_tid; idx < ROWS_CTA * (D / 8); idx += 128) {
+                const int r = idx / (D / 8);
+                const int cc = idx - r * (D / 8);
+                const int gr = ROWS_CTA * static_cast<int>(rank) + r;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (gr < args.rows) v = ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + cc * 8);
+                const uint32_t dst = base + OFF_Q + (cc >> 3) * (ROWS_CTA * 128) + sw128(r, cc & 7);
+                st_shared_v4(dst, v.x, v.y, v.z, v.w);
+            }
+            ptx::fence_proxy_async_smem();
+            arrive_leader(&misc->q_ready);
+        };
+
+        int64_t k = 0;
+        int64_t seg_no = 0;
+        bool have = walk.next();
+        if (have) load_q(walk.seg_b);
+        while (have && !*abort_flag) {
+            const int32_t seg_b = walk.seg_b;
+            const int32_t L = walk.L;
+            const int64_t slot = walk.slot;
+            const int64_t k0 = k;
+            const int64_t t_begin = walk.t_begin, t_end = walk.t_end;
+            const int32_t vis = real_row ? (L - args.n_q + qi + 1) : 0;
+            float m_run = -INFINITY;      // running max (raw score units)
+            float l_run = 0.f;            // this lane's share of the row sum
+            bool ok = true;
+            for (int64_t t = t_begin; t < t_end; ++t, ++k) {
+                const int s = static_cast<int>(k & 1);
+                if (!wait_bounded(bar(&misc->s_full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                uint32_t sr[32];
+                ptx::tmem_ld32(tmem + lane_base + TMEM_S + 32 * s, sr);
+                ptx::tmem_wait_ld();
+                ptx::tc_fence_before();
+                arrive_leader(&misc->s_free[s]);
+
+                const int32_t tok0 = static_cast<int32_t>(t) * TOK + half * OWN;
+                float v[32];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    v[j] = (tok0 + j < vis) ? __uint_as_float(sr[j]) : -INFINITY;
+                    mx = fmaxf(mx, v[j]);
+                }
+                misc->xmax[s][lt] = mx;
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(&misc->xbar[s]));
+                if (!wait_bounded(bar(&misc->xbar[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                mx = fmaxf(mx, misc->xmax[s][lt ^ 64]);
+
+                float alpha = 1.f;
+                if (mx > -INFINITY && (m_run == -INFINITY ||
+                                       (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
+                    alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - mx) * args.scale_log2);
+                    m_run = mx;
+                }
+                const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
+                float psum = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    v[j] = exp2f(fmaf(v[j], args.scale_log2, -mb));   // -inf -> 0
+                    psum += v[j];
+                }
+                l_run = fmaf(l_run, alpha, psum);
+
+                // rescale the accumulated O rows held by this lane
+                const bool need = (k > k0) && (alpha != 1.f);
+                if (__any_sync(0xffffffffu, need)) {
+                    const int64_t kp = k - 1;
+                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                      args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+#pragma unroll 1
+                    for (int cch = 0; cch < 8; ++cch) {
+                        uint32_t o[32];
+                        const uint32_t ta = tmem + lane_base + TMEM_O + 32 * cch;
+                        ptx::tmem_ld32(ta, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        ptx::tmem_st32(ta, o);
+                    }
+                    ptx::tmem_wait_st();
+                }
+                // P buffer s is free once the value product of tile k-2 is done
+                if (k >= 2) {
+                    const int64_t kp = k - 2;
+                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                      args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                const uint32_t pb = base + OFF_P + s * P_BYTES;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    st_shared_v4(pb + sw128(row, 4 * half + c),
+                                 pack_bf16x2(v[8 * c + 0], v[8 * c + 1]),
+                                 pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                 pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                                 pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                arrive_leader(&misc->p_ready[s]);
+            }
+            if (!ok) break;
+
+            // next segment's Q may be loaded now: QK^T of this segment is complete
+            have = walk.next();
+            if (have) load_q(walk.seg_b);
+
+            // epilogue of this segment
+            const int64_t kl = k - 1;
+            if (!wait_bounded(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
+                              args.timeout_ns))
+                break;
+            ptx::tc_fence_after();
+            misc->xl[lt] = l_run;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(&misc->xlbar));
+            if (!wait_bounded(bar(&misc->xlbar), seg_no & 1, abort_flag, args.timeout_ns)) break;
+            ++seg_no;
+            const float l_row = l_run + misc->xl[lt ^ 64];
+            const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
+            float *dst = args.o_part + (slot * args.rows + grow) * DC;
+#pragma unroll 1
+            for (int cch = 0; cch < 8; ++cch) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
+                ptx::tmem_wait_ld();
+                if (real_row) {
+                    // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
+                    const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + ch);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv,
+                                            __uint_as_float(o[4 * j + 1]) * inv,
+                                            __uint_as_float(o[4 * j + 2]) * inv,
+                                            __uint_as_float(o[4 * j + 3]) * inv);
+                }
+            }
+            if (real_row && half == 0) {
+                args.lse_part[slot * args.rows + grow] =
+                    (l_row > 0.f) ? m_run * args.scale + logf(l_row) : -INFINITY;
+            }
+            ptx::tc_fence_before();
+            arrive_leader(&misc->o_free);
+            (void)seg_b;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc<2>(tmem, TMEM_COLS);
+}
+
+// ===========================================================================
+// Single-CTA kernel: d_c = 64, d_R = 8 (RoPE padded to 16 in shared memory)
+// ===========================================================================
+namespace single {
+constexpr int DC = 64, DR = 8, D = DC + DR;
+constexpr int ROWS = 128;
+constexpr int TOK = 128;                        // tokens per tile (two pages)
+constexpr uint32_t Q_LAT = ROWS * 128;          // 16384: [128 rows x 64 ch] swizzled
+constexpr uint32_t Q_ROPE = ROWS * 16;          // 2048: [128 rows x 8 ch] core matrices
+constexpr uint32_t Q_BYTES = Q_LAT + 2 * Q_ROPE;          // + zero K-chunk
+constexpr uint32_t ST_LAT = TOK * 128;                    // 16384
+constexpr uint32_t ST_ROPE = TOK * 16;                    // 2048
+constexpr uint32_t STAGE_BYTES = ST_LAT + 2 * ST_ROPE;    // 20480
+constexpr int STAGES = 2;
+constexpr uint32_t P_BYTES = 2 * ROWS * 128;              // [128 rows x 128 tok] = 2 K-blocks
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_STAGE = 20480;                     // Q rounded up to 1 KB multiple
+constexpr uint32_t OFF_P = OFF_STAGE + STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + pair::MISC_BYTES + 1024;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_O = 0;                            // 64 columns
+constexpr uint32_t TMEM_S = 128;                          // two 128-column score buffers
+constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, DC, 0, 1);
+static_assert(Q_BYTES <= OFF_STAGE, "q");
+static_assert(SMEM_BYTES <= 232448, "smem");
+static_assert((OFF_P % 1024) == 0 && (OFF_MISC % 1024) == 0, "align");
+}  // namespace single
+
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_single_kernel(const __grid_constant__ CUtensorMap map_ckv,
+                         const __grid_constant__ CUtensorMap map_kr, const DecodeArgs args) {
+    using namespace single;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_base);
+    Misc *misc = reinterpret_cast<Misc *>(smem + OFF_MISC);
+    volatile int32_t *abort_flag = &misc->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t part = blockIdx.x;
+    const int64_t P = args.num_parts;
+    auto bar = [&](const uint64_t *b) { return ptx::smem_u32(b); };
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(bar(&misc->full[i]), 1);
+            ptx::mbar_init(bar(&misc->empty[i]), 1);
+            ptx::mbar_init(bar(&misc->s_full[i]), 1);
+            ptx::mbar_init(bar(&misc->s_free[i]), 4);
+            ptx::mbar_init(bar(&misc->p_ready[i]), 4);
+            ptx::mbar_init(bar(&misc->pv_done[i]), 1);
+        }
+        ptx::mbar_init(bar(&misc->q_ready), 4);
+        ptx::mbar_init(bar(&misc->o_free), 4);
+        ptx::mbar_init(bar(&misc->drain), 1);
+        misc->abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    // zero the stages and Q (so never-loaded rows and the padded RoPE K-chunk
+    // hold zeros rather than stale bit patterns)
+    for (uint32_t off = threadIdx.x * 16; off < OFF_MISC; off += kDecodeThreads * 16)
+        st_shared_v4(base + off, 0, 0, 0, 0);
+    ptx::fence_proxy_async_smem();
+    if (warp == 0) {
+        const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
+                                          P, 0);
+        const int64_t N = c.total;
+        const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
+        const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
+                                          P, ts);
+        if (lane == 0) {
+            misc->cur_b = s.b;
+            misc->cur_O = s.tile_off;
+            misc->cur_S = s.slot_base;
+            misc->cur_N = N;
+            ptx::prefetch_tensormap(&map_ckv);
+            ptx::prefetch_tensormap(&map_kr);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<1>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
+        ptx::tmem_relinquish<1>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    SegmentWalker walk;
+    walk.seq_lens = args.seq_lens;
+    walk.batch = args.batch;
+    walk.max_pages = args.max_pages;
+    walk.n_q = args.n_q;
+    walk.tile_tokens = TOK;
+    walk.N = misc->cur_N;
+    walk.P = parts_in_use(P, walk.N);
+    walk.p = part;
+    walk.b = misc->cur_b;
+    walk.O = misc->cur_O;
+    walk.S = misc->cur_S;
+    if (part < walk.P) {
+        walk.tile = part_start(part, walk.N, walk.P);
+        walk.te = part_start(part + 1, walk.N, walk.P);
+    } else {
+        walk.tile = walk.te = 0;   // idle partition
+    }
+
+    if (warp == 0) {
+        if (ptx::elect_one()) {
+            int64_t k = 0;
+            bool bad_page = false;
+            while (!*abort_flag && walk.next()) {
+                const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
+                const int32_t npages = (walk.L + 63) / 64;
+                for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
+                    const int s = static_cast<int>(k & 1);
+                    const int32_t p0 = static_cast<int32_t>(2 * t);
+                    const bool two = p0 + 1 < npages;
+                    int32_t pg[2] = {trow[p0], two ? trow[p0 + 1] : 0};
+                    for (int i = 0; i < 2; ++i)
+                        if (pg[i] < 0 || pg[i] >= args.num_pages) { bad_page = true; pg[i] = 0; }
+                    if (k >= 2 && !wait_bounded(bar(&misc->empty[s]), ((k >> 1) - 1) & 1,
+                                                abort_flag, args.timeout_ns))
+                        break;
+                    const uint32_t fb = bar(&misc->full[s]);
+                    const uint32_t npg = two ? 2u : 1u;
+                    ptx::mbar_arrive_expect_tx(fb, npg * (64 * 128 + 64 * 16));
+                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    for (uint32_t i = 0; i < npg; ++i) {
+                        ptx::tma_load_3d(st + i * (64 * 128), &map_ckv, fb, 0, 0, pg[i]);
+                        ptx::tma_load_3d(st + ST_LAT + i * (64 * 16), &map_kr, fb, 0, 0, pg[i]);
+                    }
+                }
+            }
+            if (bad_page) record_error(kErrDeviceBounds);
+            for (int64_t kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk)
+                wait_bounded(bar(&misc->full[kk & 1]), (kk >> 1) & 1, abort_flag, args.timeout_ns);
+        }
+    } else if (warp == 1) {
+        if (ptx::elect_one()) {
+            int64_t k = 0, g = 0;
+            bool ok = true;
+            auto issue_pv = [&](int64_t kp, bool first_of_seg) -> bool {
+                const int s = static_cast<int>(kp & 1);
+                if (!wait_bounded(bar(&misc->p_ready[s]), (kp >> 1) & 1, abort_flag, args.timeout_ns))
+                    return false;
+                ptx::tc_fence_after();
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint32_t pbuf = base + OFF_P + s * P_BYTES;
+                for (int kk = 0; kk < TOK / 16; ++kk) {
+                    const uint64_t a = ptx::smem_desc(pbuf + (kk >> 2) * (ROWS * 128) + (kk & 3) * 32,
+                                                      16, 1024, ptx::kSwizzle128B);
+                    const uint64_t b = ptx::smem_desc(st + kk * 2048, 8192, 1024, ptx::kSwizzle128B);
+                    ptx::mma_bf16_ss<1>(tmem + TMEM_O, a, b, IDESC_PV,
+                                        (first_of_seg && kk == 0) ? 0u : 1u);
+                }
+                ptx::mma_commit(bar(&misc->empty[s]));
+                ptx::mma_commit(bar(&misc->pv_done[s]));
+                return true;
+            };
+            while (ok && !*abort_flag && walk.next()) {
+                const int64_t k0 = k;
+                if (!wait_bounded(bar(&misc->q_ready), g & 1, abort_flag, args.timeout_ns)) break;
+                for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
+                    const int s = static_cast<int>(k & 1);
+                    if (!wait_bounded(bar(&misc->full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (k >= 2 && !wait_bounded(bar(&misc->s_free[s]), ((k >> 1) - 1) & 1,
+                                                abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a = ptx::smem_desc(base + OFF_Q + kk * 32, 16, 1024,
+                                                          ptx::kSwizzle128B);
+                        const uint64_t b = ptx::smem_desc(st + kk * 32, 16, 1024, ptx::kSwizzle128B);
+                        ptx::mma_bf16_ss<1>(tmem + TMEM_S + TOK * s, a, b, IDESC_QK, kk ? 1u : 0u);
+                    }
+                    {   // RoPE step: 8 real channels + 8 zero channels, no swizzle
+                        const uint64_t a = ptx::smem_desc(base + OFF_Q + Q_LAT, Q_ROPE, 128,
+                                                          ptx::kSwizzleNone);
+                        const uint64_t b = ptx::smem_desc(st + ST_LAT, ST_ROPE, 128, ptx::kSwizzleNone);
+                        ptx::mma_bf16_ss<1>(tmem + TMEM_S + TOK * s, a, b, IDESC_QK, 1u);
+                    }
+                    ptx::mma_commit(bar(&misc->s_full[s]));
+                    if (k > k0) {
+                        if (k - 1 == k0 && g > 0) {
+                            if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag,
+                                              args.timeout_ns)) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!issue_pv(k - 1, k - 1 == k0)) { ok = false; break; }
+                    }
+                }
+                if (!ok) break;
+                if (k - 1 == k0 && g > 0) {
+                    if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag, args.timeout_ns))
+                        break;
+                }
+                if (!issue_pv(k - 1, k - 1 == k0)) break;
+                ++g;
+            }
+            ptx::mma_commit(bar(&misc->drain));
+            wait_bounded(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
+        }
+    } else {
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;                 // query row = TMEM lane
+        const bool real_row = row < args.rows;
+        const bool warp_real = (q4 * 32) < args.rows;   // warp holds at least one real row
+        const int qi = real_row ? row / args.heads : 0;
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const int st_tid = threadIdx.x - kSoftmaxWarp0 * 32;
+        auto arrive = [&](uint64_t *b) {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(b));
+        };
+        auto load_q = [&](int32_t b) {
+            const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
+            for (int idx = st_tid; idx < ROWS * (D / 8); idx += 128) {
+                const int r = idx / (D / 8);
+                const int cc = idx - r * (D / 8);
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (r < args.rows) v = ld_global_nc_v4(qb + static_cast<int64_t>(r) * D + cc * 8);
+                uint32_t dst;
+                if (cc < 8) dst = base + OFF_Q + sw128(r, cc);
+                else dst = base + OFF_Q + Q_LAT + (r >> 3) * 128 + (r & 7) * 16;
+                st_shared_v4(dst, v.x, v.y, v.z, v.w);
+            }
+            ptx::fence_proxy_async_smem();
+            arrive(&misc->q_ready);
+        };
+
+        int64_t k = 0;
+        bool have = walk.next();
+        if (have) load_q(walk.seg_b);
+        while (have && !*abort_flag) {
+            const int32_t L = walk.L;
+            const int64_t slot = walk.slot;
+            const int64_t k0 = k;
+            const int64_t t_begin = walk.t_begin, t_end = walk.t_end;
+            const int32_t vis = real_row ? (L - args.n_q + qi + 1) : 0;
+            float m_run = -INFINITY, l_run = 0.f;
+            bool ok = true;
+            for (int64_t t = t_begin; t < t_end; ++t, ++k) {
+                const int s = static_cast<int>(k & 1);
+                if (!wait_bounded(bar(&misc->s_full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                float v[TOK];
+                if (warp_real) {
+#pragma unroll
+                    for (int c = 0; c < TOK / 32; ++c) {
+                        uint32_t sr[32];
+                        ptx::tmem_ld32(tmem + lane_base + TMEM_S + TOK * s + 32 * c, sr);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[32 * c + j] = __uint_as_float(sr[j]);
+                    }
+                }
+                ptx::tc_fence_before();
+                arrive(&misc->s_free[s]);
+
+                float alpha = 1.f;
+                if (warp_real) {
+                    const int32_t tok0 = static_cast<int32_t>(t) * TOK;
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < TOK; ++j) {
+                        v[j] = (tok0 + j < vis) ? v[j] : -INFINITY;
+                        mx = fmaxf(mx, v[j]);
+                    }
+                    if (mx > -INFINITY && (m_run == -INFINITY ||
+                                           (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
+                        alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - mx) * args.scale_log2);
+                        m_run = mx;
+                    }
+                    const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
+                    float psum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < TOK; ++j) {
+                        v[j] = exp2f(fmaf(v[j], args.scale_log2, -mb));
+                        psum += v[j];
+                    }
+                    l_run = fmaf(l_run, alpha, psum);
+                }
+                const bool need = warp_real && (k > k0) && (alpha != 1.f);
+                if (__any_sync(0xffffffffu, need)) {
+                    const int64_t kp = k - 1;
+                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                      args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+#pragma unroll 1
+                    for (int cch = 0; cch < DC / 32; ++cch) {
+                        uint32_t o[32];
+                        const uint32_t ta = tmem + lane_base + TMEM_O + 32 * cch;
+                        ptx::tmem_ld32(ta, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        ptx::tmem_st32(ta, o);
+                    }
+                    ptx::tmem_wait_st();
+                }
+                if (k >= 2) {
+                    const int64_t kp = k - 2;
+                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                      args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (warp_real) {
+                    const uint32_t pb = base + OFF_P + s * P_BYTES;
+#pragma unroll
+                    for (int c = 0; c < TOK / 8; ++c) {
+                        st_shared_v4(pb + (c >> 3) * (ROWS * 128) + sw128(row, c & 7),
+                                     pack_bf16x2(v[8 * c + 0], v[8 * c + 1]),
+                                     pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                     pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                                     pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+                    }
+                    ptx::fence_proxy_async_smem();
+                }
+                ptx::tc_fence_before();
+                arrive(&misc->p_ready[s]);
+            }
+            if (!ok) break;
+            have = walk.next();
+            if (have) load_q(walk.seg_b);
+            const int64_t kl = k - 1;
+            if (!wait_bounded(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
+                              args.timeout_ns))
+                break;
+            ptx::tc_fence_after();
+            if (warp_real) {
+                const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                float *dst = args.o_part + (slot * args.rows + row) * DC;
+#pragma unroll 1
+                for (int cch = 0; cch < DC / 32; ++cch) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
+                    ptx::tmem_wait_ld();
+                    if (real_row) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cch);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv,
+                                                __uint_as_float(o[4 * j + 1]) * inv,
+                                                __uint_as_float(o[4 * j + 2]) * inv,
+                                                __uint_as_float(o[4 * j + 3]) * inv);
+                    }
+                }
+                if (real_row)
+                    args.lse_part[slot * args.rows + row] =
+                        (l_run > 0.f) ? m_run * args.scale + logf(l_run) : -INFINITY;
+            }
+            ptx::tc_fence_before();
+            arrive(&misc->o_free);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc<1>(tmem, TMEM_COLS);
+}
+
+}  // namespace mla

@@ -1,0 +1,378 @@
+// Host side of the C ABI declared in include/mla_decode.h: argument
+// validation, tensor-map construction, the partition plan and kernel launches.
+// Everything is asynchronous on the caller's stream; no device memory is
+// allocated here.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mla_decode.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "small_kernels.cuh"
+
+namespace {
+
+using mla::kErrCuda;
+using mla::kErrInvalidArg;
+using mla::kErrUnsupported;
+
+constexpr int64_t kDefaultTimeoutNs = 2000000000LL;   // 2 s per bounded wait
+constexpr int kMaxDevices = 64;
+
+enum class Variant { Pair512, Single64, None };
+
+Variant variant_of(const mla_dims *d) {
+    if (d->d_latent == 512 && d->d_rope == 64) return Variant::Pair512;
+    if (d->d_latent == 64 && d->d_rope == 8) return Variant::Single64;
+    return Variant::None;
+}
+
+int tile_tokens(Variant v) { return v == Variant::Pair512 ? mla::pair::TOK : mla::single::TOK; }
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validates the dims common to every call; returns MLA_OK or an error.
+mla_status check_dims(const mla_dims *d, bool need_variant) {
+    if (!d) return MLA_ERR_INVALID_ARG;
+    if (d->num_heads <= 0 || d->n_q <= 0 || d->d_nope <= 0 || d->d_latent <= 0 || d->d_rope <= 0 ||
+        d->d_v <= 0 || d->page_size <= 0)
+        return MLA_ERR_INVALID_ARG;
+    if ((d->d_nope % 8) || (d->d_latent % 8) || (d->d_rope % 8) || (d->d_v % 8))
+        return MLA_ERR_UNSUPPORTED;
+    if (need_variant) {
+        if (variant_of(d) == Variant::None) return MLA_ERR_UNSUPPORTED;
+        if (d->page_size != 64) return MLA_ERR_UNSUPPORTED;
+        if (static_cast<int64_t>(d->n_q) * d->num_heads > 128) return MLA_ERR_UNSUPPORTED;
+    }
+    return MLA_OK;
+}
+
+float scale_of(const mla_dims *d) {
+    return d->softmax_scale > 0.f ? d->softmax_scale
+                                  : static_cast<float>(1.0 / std::sqrt(double(d->d_nope + d->d_rope)));
+}
+
+// Per-device one-time state: capability check and kernel attributes.
+struct DeviceState {
+    std::once_flag once;
+    mla_status status = MLA_OK;
+};
+DeviceState g_dev[kMaxDevices];
+
+mla_status device_ready() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    DeviceState &st = g_dev[dev];
+    std::call_once(st.once, [&] {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { st.status = MLA_ERR_CUDA; return; }
+        if (prop.major != 10 || prop.minor != 0) { st.status = MLA_ERR_UNSUPPORTED; return; }
+        if (cudaFuncSetAttribute(mla::decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::pair::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_single_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::single::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::head_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::kProjTok * 512 * 4) != cudaSuccess) {
+            st.status = MLA_ERR_CUDA;
+            return;
+        }
+    });
+    return st.status;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 map over a page pool: dims (channels, 64 tokens, pages).
+mla_status pool_map(CUtensorMap *m, const mla_pool *pool, int32_t channels, int32_t num_pages,
+                    uint32_t box_ch, uint32_t box_tok, CUtensorMapSwizzle sw) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(channels), 64,
+                                static_cast<cuuint64_t>(num_pages)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pool->token_stride) * 2,
+                                   static_cast<cuuint64_t>(pool->page_stride) * 2};
+    const cuuint32_t box[3] = {box_ch, box_tok, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool->base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
+}
+
+mla_status check_pool(const mla_pool *p, int32_t channels) {
+    if (!p || !p->base) return MLA_ERR_INVALID_ARG;
+    if (!aligned(p->base, 16)) return MLA_ERR_INVALID_ARG;
+    if (p->token_stride < channels || p->page_stride < p->token_stride) return MLA_ERR_INVALID_ARG;
+    if ((p->token_stride % 8) || (p->page_stride % 8)) return MLA_ERR_INVALID_ARG;
+    return MLA_OK;
+}
+
+mla_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char *mla_status_string(int32_t s) {
+    switch (s) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+        case MLA_ERR_DEVICE_BOUNDS: return "MLA_ERR_DEVICE_BOUNDS";
+        case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+        default: return "MLA_ERR_UNKNOWN";
+    }
+}
+
+int32_t mla_decode_num_parts(const mla_dims *dims, int64_t total_tiles, int32_t num_sms) {
+    if (check_dims(dims, true) != MLA_OK || num_sms <= 0) return 1;
+    const Variant v = variant_of(dims);
+    const int64_t units = (v == Variant::Pair512) ? num_sms / 2 : num_sms;
+    const int64_t min_tiles = (v == Variant::Pair512) ? 8 : 4;
+    int64_t parts = (total_tiles + min_tiles - 1) / min_tiles;
+    if (parts > units) parts = units;
+    if (parts < 1) parts = 1;
+    return static_cast<int32_t>(parts);
+}
+
+size_t mla_decode_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t num_parts) {
+    if (check_dims(dims, true) != MLA_OK || batch < 0 || num_parts <= 0) return 0;
+    const int64_t slots = static_cast<int64_t>(batch) + num_parts;
+    const int64_t R = static_cast<int64_t>(dims->n_q) * dims->num_heads;
+    const int64_t o_bytes = round_up(slots * R * dims->d_latent * 4, 256);
+    return static_cast<size_t>(o_bytes + round_up(slots * R * 4, 256));
+}
+
+int64_t mla_decode_plan(const mla_dims *dims, const int32_t *seq_lens_host,
+                        int32_t max_pages_per_seq, int32_t batch, int32_t num_parts,
+                        int32_t *part_first, int32_t *slot_count, int64_t *slot_base) {
+    if (check_dims(dims, true) != MLA_OK || batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0)
+        return -1;
+    if (batch > 0 && !seq_lens_host) return -1;
+    const int T = tile_tokens(variant_of(dims));
+    int64_t N = 0;
+    bool bad = false;
+    for (int32_t b = 0; b < batch; ++b)
+        N += mla::tiles_of_len(mla::clamp_len(seq_lens_host[b], max_pages_per_seq, dims->n_q, &bad), T);
+    const int64_t P = mla::parts_in_use(num_parts, N);
+    int64_t O = 0, S = 0;
+    for (int32_t b = 0; b < batch; ++b) {
+        const int64_t n =
+            mla::tiles_of_len(mla::clamp_len(seq_lens_host[b], max_pages_per_seq, dims->n_q, &bad), T);
+        int64_t pf = -1, cnt = 0;
+        if (n > 0) {
+            pf = mla::part_of_tile(O, N, P);
+            cnt = mla::part_of_tile(O + n - 1, N, P) - pf + 1;
+        }
+        if (part_first) part_first[b] = static_cast<int32_t>(pf);
+        if (slot_count) slot_count[b] = static_cast<int32_t>(cnt);
+        if (slot_base) slot_base[b] = S;
+        S += cnt;
+        O += n;
+    }
+    return S;
+}
+
+mla_status mla_absorb_q(const mla_dims *dims, const void *q_c, const void *q_r, const void *w_uk,
+                        void *q_out, int32_t num_tokens, void *stream) {
+    mla_status st = check_dims(dims, false);
+    if (st != MLA_OK) return st;
+    if (num_tokens < 0) return MLA_ERR_INVALID_ARG;
+    if (dims->d_nope > 512) return MLA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return MLA_OK;
+    if (!q_c || !q_r || !w_uk || !q_out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q_c, 16) || !aligned(q_r, 16) || !aligned(w_uk, 16) || !aligned(q_out, 16))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    mla::ProjArgs a;
+    a.x = static_cast<const __nv_bfloat16 *>(q_c);
+    a.w = static_cast<const __nv_bfloat16 *>(w_uk);
+    a.out = static_cast<__nv_bfloat16 *>(q_out);
+    a.rope = static_cast<const __nv_bfloat16 *>(q_r);
+    a.T = num_tokens;
+    a.H = dims->num_heads;
+    a.K = dims->d_nope;
+    a.n_cols = dims->d_latent;
+    a.out_stride = dims->d_latent + dims->d_rope;
+    a.d_rope = dims->d_rope;
+    dim3 grid(dims->num_heads, (dims->d_latent + 127) / 128, (num_tokens + mla::kProjTok - 1) / mla::kProjTok);
+    mla::head_proj_kernel<<<grid, 128, mla::kProjTok * a.K * 4, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w_uv, void *out,
+                          int32_t num_tokens, void *stream) {
+    mla_status st = check_dims(dims, false);
+    if (st != MLA_OK) return st;
+    if (num_tokens < 0) return MLA_ERR_INVALID_ARG;
+    if (dims->d_latent > 512) return MLA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return MLA_OK;
+    if (!o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(o_lat, 16) || !aligned(w_uv, 16) || !aligned(out, 16)) return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    mla::ProjArgs a;
+    a.x = static_cast<const __nv_bfloat16 *>(o_lat);
+    a.w = static_cast<const __nv_bfloat16 *>(w_uv);
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.rope = nullptr;
+    a.T = num_tokens;
+    a.H = dims->num_heads;
+    a.K = dims->d_latent;
+    a.n_cols = dims->d_v;
+    a.out_stride = dims->d_v;
+    a.d_rope = 0;
+    dim3 grid(dims->num_heads, (dims->d_v + 127) / 128, (num_tokens + mla::kProjTok - 1) / mla::kProjTok);
+    mla::head_proj_kernel<<<grid, 128, mla::kProjTok * a.K * 4, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_pool *ckv,
+                              const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                              int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                              int32_t num_parts, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0 || num_pages <= 0)
+        return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!q || !block_table || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+        !aligned(workspace, 256))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    if (workspace_bytes < mla_decode_workspace_bytes(dims, batch, num_parts)) return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+
+    const int64_t R = static_cast<int64_t>(dims->n_q) * dims->num_heads;
+    const int64_t slots = static_cast<int64_t>(batch) + num_parts;
+    mla::DecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.o_part = static_cast<float *>(workspace);
+    a.lse_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                           round_up(slots * R * dims->d_latent * 4, 256));
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.max_pages = max_pages_per_seq;
+    a.batch = batch;
+    a.num_pages = num_pages;
+    a.num_parts = num_parts;
+    a.n_q = dims->n_q;
+    a.heads = dims->num_heads;
+    a.rows = static_cast<int32_t>(R);
+    a.scale = scale_of(dims);
+    a.scale_log2 = a.scale * 1.4426950408889634f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (variant_of(dims) == Variant::Pair512) {
+        CUtensorMap m32, m64, mkr;
+        if ((st = pool_map(&m32, ckv, 512, num_pages, 64, mla::pair::OWN,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+            return st;
+        if ((st = pool_map(&m64, ckv, 512, num_pages, 64, mla::pair::TOK,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+            return st;
+        if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+            return st;
+        mla::decode_pair_kernel<<<2 * num_parts, mla::kDecodeThreads, mla::pair::SMEM_BYTES, s>>>(
+            m32, m64, mkr, a);
+    } else {
+        CUtensorMap mc, mkr;
+        if ((st = pool_map(&mc, ckv, 64, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+            return st;
+        if ((st = pool_map(&mkr, kr, 8, num_pages, 8, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != MLA_OK)
+            return st;
+        mla::decode_single_kernel<<<num_parts, mla::kDecodeThreads, mla::single::SMEM_BYTES, s>>>(
+            mc, mkr, a);
+    }
+    return launch_status();
+}
+
+mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t workspace_bytes,
+                       const int32_t *seq_lens, int32_t max_pages_per_seq, int32_t batch,
+                       int32_t num_parts, void *o_lat, float *lse_out, void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!workspace || !seq_lens || !o_lat) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(o_lat, 16) || !aligned(seq_lens, 4) ||
+        (lse_out && !aligned(lse_out, 4)))
+        return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_decode_workspace_bytes(dims, batch, num_parts)) return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    const int64_t R = static_cast<int64_t>(dims->n_q) * dims->num_heads;
+    const int64_t slots = static_cast<int64_t>(batch) + num_parts;
+    mla::CombineArgs a;
+    a.o_part = static_cast<const float *>(workspace);
+    a.lse_part = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) +
+                                                 round_up(slots * R * dims->d_latent * 4, 256));
+    a.seq_lens = seq_lens;
+    a.o_lat = static_cast<__nv_bfloat16 *>(o_lat);
+    a.lse_out = lse_out;
+    a.batch = batch;
+    a.max_pages = max_pages_per_seq;
+    a.n_q = dims->n_q;
+    a.rows = static_cast<int32_t>(R);
+    a.d_c = dims->d_latent;
+    a.tile_tokens = tile_tokens(variant_of(dims));
+    a.num_parts = num_parts;
+    dim3 grid(batch, static_cast<unsigned>((R + 3) / 4));
+    mla::combine_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+mla_status mla_get_device_error(int32_t *code, void *stream) {
+    if (!code) return MLA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, mla::g_device_error, sizeof(v)) != cudaSuccess) return MLA_ERR_CUDA;
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(mla::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return MLA_ERR_CUDA;
+    *code = v;
+    return MLA_OK;
+}
+
+mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream) {
+    if (timeout_ns <= 0) return MLA_ERR_INVALID_ARG;
+    mla_status st = device_ready();
+    if (st != MLA_OK) return st;
+    mla::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and its host-side logic (partition plan, workspace sizing,
+argument validation) behaves as documented. No kernel is launched here."""
+import ctypes
+import os
+import random
+import re
+
+import pytest
+import torch
+
+from mla_latent_kv_18_b200 import build as mla_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def b():
+    mla_build.build()
+    from mla_latent_kv_18_b200 import _binding
+    return _binding
+
+
+def _declared():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(b):
+    declared = _declared()
+    assert {"mla_absorb_q", "mla_decode_splitkv", "mla_combine", "mla_absorb_out"} <= declared
+    for name in declared:
+        assert hasattr(b.lib, name), name
+    assert set(b.EXPORTS) == declared
+
+
+def test_status_strings(b):
+    for code, name in b.STATUS_NAMES.items():
+        assert b.lib.mla_status_string(code).decode() == name
+    assert b.lib.mla_status_string(99).decode() == "MLA_ERR_UNKNOWN"
+
+
+def _dims(b, **kw):
+    d = dict(num_heads=128, n_q=1, d_nope=128, d_latent=512, d_rope=64, d_v=128, page_size=64,
+             softmax_scale=0.0)
+    d.update(kw)
+    return b.MLADims(**d)
+
+
+def _brute_plan(lens, max_pages, n_q, T, P):
+    n = []
+    for L in lens:
+        L = max(0, min(L, max_pages * 64))
+        n.append((L + T - 1) // T)
+    N = sum(n)
+    P = min(P, N) if N else P
+    owner = []
+    for p in range(P):
+        owner += [p] * ((p + 1) * N // P - p * N // P)
+    assert len(owner) == N
+    off, base = 0, 0
+    first, count, bases = [], [], []
+    for nb in n:
+        parts = sorted(set(owner[off:off + nb]))
+        first.append(parts[0] if parts else -1)
+        count.append(len(parts))
+        bases.append(base)
+        base += len(parts)
+        off += nb
+    return first, count, bases, base
+
+
+@pytest.mark.parametrize("latent", [512, 64])
+def test_plan_matches_brute_force(b, latent):
+    from mla_latent_kv_18_b200 import api
+    rng = random.Random(0)
+    dims = _dims(b, d_latent=latent, d_rope=64 if latent == 512 else 8,
+                 num_heads=128 if latent == 512 else 32, n_q=1 if latent == 512 else 2)
+    T = 64 if latent == 512 else 128
+    for trial in range(200):
+        B = rng.randint(1, 40)
+        max_pages = rng.randint(1, 40)
+        lens = [rng.randint(dims.n_q, max_pages * 64) for _ in range(B)]
+        P = rng.randint(1, 80)
+        pf, cnt, base, total = api.plan(dims, lens, max_pages, P)
+        e_first, e_cnt, e_base, e_total = _brute_plan(lens, max_pages, dims.n_q, T, P)
+        assert pf.tolist() == e_first and cnt.tolist() == e_cnt and base.tolist() == e_base
+        assert total == e_total <= B + P - 1
+
+
+def test_num_parts_and_workspace(b):
+    d = _dims(b)
+    lib = b.lib
+    assert lib.mla_decode_num_parts(ctypes.byref(d), 4, 148) == 1
+    assert lib.mla_decode_num_parts(ctypes.byref(d), 16 * 1024, 148) == 74
+    assert lib.mla_decode_num_parts(ctypes.byref(d), 0, 148) == 1
+    ws = lib.mla_decode_workspace_bytes(ctypes.byref(d), 16, 74)
+    slots, R = 16 + 74, 128
+    o = (slots * R * 512 * 4 + 255) // 256 * 256
+    assert ws == o + (slots * R * 4 + 255) // 256 * 256
+    bad = _dims(b, d_latent=256)
+    assert lib.mla_decode_workspace_bytes(ctypes.byref(bad), 16, 74) == 0
+
+
+def test_argument_validation_without_launch(b):
+    lib = b.lib
+    d = _dims(b)
+    null = ctypes.c_void_p(0)
+    pool = b.MLAPool(0, 64 * 512, 512)
+    # batch 0 is a no-op, checked before anything touches a device
+    assert lib.mla_decode_splitkv(ctypes.byref(d), null, ctypes.byref(pool), ctypes.byref(pool),
+                                  1, null, 1, null, 0, 1, null, 0, null) == 0
+    # null pointers with work to do
+    assert lib.mla_decode_splitkv(ctypes.byref(d), null, ctypes.byref(pool), ctypes.byref(pool),
+                                  1, null, 1, null, 2, 1, null, 0, null) == 1
+    # unsupported latent width
+    d2 = _dims(b, d_latent=256)
+    assert lib.mla_decode_splitkv(ctypes.byref(d2), null, ctypes.byref(pool), ctypes.byref(pool),
+                                  1, null, 1, null, 2, 1, null, 0, null) == 2
+    # too many query rows per sequence
+    d3 = _dims(b, n_q=2)
+    assert lib.mla_combine(ctypes.byref(d3), null, 0, null, 1, 2, 1, null, null, null) == 2
+    # misaligned pointers are rejected before any launch
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1002)
+    assert lib.mla_absorb_q(ctypes.byref(d), odd, fake, fake, fake, 4, null) == 1
+    assert lib.mla_absorb_out(ctypes.byref(d), fake, odd, fake, 4, null) == 1
+    assert lib.mla_absorb_q(ctypes.byref(d), fake, fake, fake, fake, -1, null) == 1
+    assert lib.mla_absorb_q(ctypes.byref(d), null, null, null, null, 0, null) == 0
+    ws_bytes = lib.mla_decode_workspace_bytes(ctypes.byref(d), 2, 1)
+    bad_pool = b.MLAPool(0x1000, 64 * 512, 500)          # token stride below the width
+    assert lib.mla_decode_splitkv(ctypes.byref(d), fake, ctypes.byref(bad_pool),
+                                  ctypes.byref(bad_pool), 1, fake, 1, fake, 2, 1,
+                                  ctypes.c_void_p(0x10000), ws_bytes, null) == 1
+    good = b.MLAPool(0x1000, 64 * 576, 576)
+    assert lib.mla_decode_splitkv(ctypes.byref(d), fake, ctypes.byref(good), ctypes.byref(good),
+                                  1, fake, 1, fake, 2, 1, ctypes.c_void_p(0x10000), ws_bytes - 4,
+                                  null) == 1                # workspace too small
+    assert lib.mla_decode_splitkv(ctypes.byref(d), fake, ctypes.byref(good), ctypes.byref(good),
+                                  1, fake, 1, fake, 2, 1, ctypes.c_void_p(0x10010), ws_bytes,
+                                  null) == 1                # workspace not 256-byte aligned
+    assert lib.mla_debug_wait_timeout(0, null) == 1
