@@ -152,9 +152,11 @@ __global__ void __launch_bounds__(128) head_proj_kernel(const ProjArgs a) {
 #pragma unroll
             for (int t = 0; t < kProjTok; ++t) acc[t] = fmaf(xs[t * a.K + k], wv, acc[t]);
         }
-        for (int t = 0; t < nt; ++t)
-            a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + col] =
-                __float2bfloat16_rn(acc[t]);
+#pragma unroll
+        for (int t = 0; t < kProjTok; ++t)
+            if (t < nt)
+                a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + col] =
+                    __float2bfloat16_rn(acc[t]);
     }
     if (a.rope && blockIdx.y == 0) {
         for (int i = threadIdx.x; i < nt * a.d_rope; i += 128) {

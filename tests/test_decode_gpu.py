@@ -41,6 +41,26 @@ def _check(got, ref, what, max_abs=MAX_ABS, rel_l2=REL_L2):
     return err, rel
 
 
+def _check_rounded(got, ref, what):
+    """Intermediate rounded to bf16 (round to nearest even): each element within one bf16 ulp
+    (2^-7 relative) of the fp64 value, plus the output bar on relative L2."""
+    got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), what
+    bound = 2.0 ** -7 * np.abs(ref) + 1e-3
+    worst = (np.abs(got - ref) / bound).max()
+    rel = np.linalg.norm((got - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-30)
+    assert worst <= 1.0 and rel <= REL_L2, f"{what}: worst err/bound {worst:.3f}, rel L2 {rel:.3e}"
+
+
+def _check_out(got, ref, what):
+    """Output bar for large-magnitude outputs: |err| <= 1e-2 + 2^-7 |ref| and rel L2 <= 5e-3."""
+    got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), what
+    worst = (np.abs(got - ref) / (MAX_ABS + 2.0 ** -7 * np.abs(ref))).max()
+    rel = np.linalg.norm((got - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-30)
+    assert worst <= 1.0 and rel <= REL_L2, f"{what}: worst err/bound {worst:.3f}, rel L2 {rel:.3e}"
+
+
 def _run(api, inp_d, num_parts=None):
     dims = api.dims_for(inp_d["q_c"], inp_d["q_r"], inp_d["w_uk"], inp_d["w_uv"])
     T = api.tile_tokens(dims)
@@ -74,7 +94,7 @@ def _parity(api, w, n_rows, n_def_rows, seed=0):
     D = w.d_latent
     # absorb-in: latent part vs fp64, RoPE part bit-exact copy
     q_ref = oracle.absorb_q(inp["q_c"], inp["w_uk"])
-    _check(_f64(r["q"][..., :D]), q_ref, "absorb_q")
+    _check_rounded(_f64(r["q"][..., :D]), q_ref, "absorb_q")
     assert torch.equal(r["q"][..., D:].cpu(), inp["q_r"])
     # split-KV + combine on the GPU's own bf16 Q (sampled rows)
     sel = _sample_rows(w, n_rows, seed)
@@ -157,14 +177,19 @@ def test_partials_match_oracle_windows(api, name, parts):
 @pytest.mark.parametrize("name,parts", [("dsv3", None), ("dsv3", 1), ("dsv3", 74),
                                         ("retrofit", None), ("retrofit", 148)])
 def test_edge_lengths(api, name, parts):
-    lens = [1, 2, 63, 64, 65, 127, 128, 129, 200, 2]
+    # lengths must be >= n_q (1 for dsv3, 2 for the causal pair of retrofit)
+    lens = [1, 2, 63, 64, 65, 127, 128, 129, 200, 3] if name == "dsv3" else \
+        [2, 3, 63, 64, 65, 127, 128, 129, 200, 2]
     w = workload(name, batch=len(lens), heads=16 if name == "dsv3" else 32, seq_len=256)
     inp = make_inputs(w, seed=5, seq_lens=lens)
     r = _run(api, to_device(inp, "cuda"), num_parts=parts)
     args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
                              "w_uk", "w_uv")]
     ab, o_lat, lse = oracle.decode_absorbed(*args)
-    _check(_f64(r["out"]), ab, "out")
+    # short sequences average few values, so outputs reach |x| ~ 4 where the bf16
+    # rounding of the output alone exceeds 1e-2: bound each element by 1e-2 plus
+    # one bf16 ulp of its value
+    _check_out(_f64(r["out"]), ab, "out")
     scale = oracle.default_scale(w.d_nope, w.d_rope)
     o_ref, lse_ref = oracle.attend_latent(r["q"].cpu(), inp["ckv_pool"], inp["kr_pool"],
                                           inp["block_table"], inp["seq_lens"], scale)
