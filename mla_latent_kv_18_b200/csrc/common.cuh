@@ -28,12 +28,41 @@ __device__ __forceinline__ void record_error(int32_t code) {
 // Bounded wait on phase `parity` of the barrier at shared address `bar`.
 // Polls the CTA's abort flag and the global timer; after `timeout_ns` it
 // records kErrTimeout, raises the abort flag and returns false.
+// kClusterScope: acquire at cluster scope (needed when another CTA's arrivals
+// publish generic-proxy data); otherwise CTA scope.
+template <bool kClusterScope = true>
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int32_t *abort_flag, int64_t timeout_ns) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    auto probe = [&] {
+        return kClusterScope ? ptx::mbar_try_wait(bar, parity) : ptx::mbar_try_wait_cta(bar, parity);
+    };
+    if (probe()) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (probe()) return true;
+        if ((it & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (static_cast<int64_t>(ptx::globaltimer_ns() - t0) > timeout_ns) {
+                record_error(kErrTimeout);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded spin until the shared-memory word at `slot` carries `tag` in its low
+// 8 bits; the word is returned in *out. False after a timeout (abort raised).
+__device__ __forceinline__ bool wait_word(const uint32_t *slot, uint32_t tag,
+                                          volatile int32_t *abort_flag, int64_t timeout_ns,
+                                          uint32_t *out) {
+    const volatile uint32_t *vs = slot;
+    uint32_t v = *vs;
+    if ((v & 0xFFu) == tag) { *out = v; return true; }
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        v = *vs;
+        if ((v & 0xFFu) == tag) { *out = v; return true; }
         if ((it & 15u) == 0u) {
             if (*abort_flag) return false;
             if (static_cast<int64_t>(ptx::globaltimer_ns() - t0) > timeout_ns) {

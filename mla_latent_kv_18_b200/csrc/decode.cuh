@@ -52,7 +52,8 @@ struct DecodeArgs {
     float scale_log2;            // scale * log2(e)
 };
 
-constexpr int kDecodeThreads = 192;          // 6 warps
+constexpr int kDecodeThreads = 192;          // single kernel: 6 warps
+constexpr int kPairThreads = 224;            // pair kernel: 7 warps (warp 6 = P.V-stage producer)
 constexpr int kSoftmaxWarp0 = 2;             // warps 2..5
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when max grows > 2^8
 
@@ -130,50 +131,55 @@ constexpr int ROWS_CTA = 64;                  // query rows per SM
 constexpr int TOK = 64;                       // tokens per tile (one page)
 constexpr int OWN = 32;                       // tokens per SM in QK^T
 constexpr uint32_t Q_BYTES = NB * ROWS_CTA * 128;           // 73728
-constexpr uint32_t STAGE_QK = NB * OWN * 128;               // 36864
-constexpr uint32_t STAGE_PV = 4 * TOK * 128;                // 32768 (4 channel blocks x 64 tokens)
-constexpr uint32_t STAGE_BYTES = STAGE_QK + STAGE_PV;       // 69632
-constexpr int STAGES = 2;
+constexpr uint32_t STAGE_QK = NB * OWN * 128;               // 36864: own 32 tokens x 9 blocks
+constexpr uint32_t STAGE_PV = 4 * TOK * 128;                // 32768: 64 tokens x this SM's 4 blocks
+constexpr int STAGES = 2;                                   // slots in each of the two rings
 constexpr uint32_t P_BYTES = ROWS_CTA * 128;                // 64 rows x 64 tokens bf16
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_STAGE = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_P = OFF_STAGE + STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_QK = OFF_Q + Q_BYTES;                // QK^T ring
+constexpr uint32_t OFF_PV = OFF_QK + STAGES * STAGE_QK;     // P.V ring
+constexpr uint32_t OFF_P = OFF_PV + STAGES * STAGE_PV;
 constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 229376
-constexpr uint32_t MISC_BYTES = 2048;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-constexpr uint32_t TX_PER_CTA = STAGE_BYTES;
+constexpr int PREFETCH = 4;                                 // L2 prefetch distance in tiles
+constexpr uint32_t MISC_BYTES = 3072;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES;   // dynamic smem base is 1 KB aligned
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
 constexpr uint32_t TMEM_S = 256;               // two 32-column score buffers
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, 256, 0, 1);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((OFF_STAGE % 1024) == 0 && (OFF_P % 1024) == 0 && (OFF_MISC % 1024) == 0, "align");
+static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 0 &&
+                  (OFF_MISC % 1024) == 0, "align");
 }  // namespace pair
 
 // misc-region layout (both kernels)
 struct Misc {
     uint64_t full[2], empty[2], s_full[2], s_free[2], p_ready[2], pv_done[2], q_ready, o_free;
-    uint64_t xbar[2], xlbar, drain;   // row-statistics exchange among softmax warps; MMA drain
+    uint64_t drain;                   // MMA drain before tensor memory is freed
+    uint64_t qk_full[2], qk_empty[2], pv_full[2], pv_empty[2];   // the pair kernel's two rings
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t cur_b;
     int32_t pad0;
     int64_t cur_O, cur_S, cur_N;
-    float xmax[2][128];
-    float xl[128];
+    uint32_t xtag[2][128];            // pair kernel: tagged half-row maxima, by tile parity
+    uint32_t xltag[128];              // pair kernel: tagged half-row sums, per segment
 };
 static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     decode_pair_kernel(const __grid_constant__ CUtensorMap map_ckv32,
                        const __grid_constant__ CUtensorMap map_ckv64,
                        const __grid_constant__ CUtensorMap map_kr32, const DecodeArgs args) {
     using namespace pair;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_base = ptx::smem_u32(smem_raw);
-    const uint32_t base = (raw_base + 1023u) & ~1023u;
-    uint8_t *smem = smem_raw + (base - raw_base);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = ptx::smem_u32(smem_raw);
+    if (base & 1023u) {   // swizzled operands need a 1 KB aligned base; uniform over the cluster
+        if (threadIdx.x == 0) record_error(kErrUnsupported);
+        return;
+    }
+    uint8_t *smem = smem_raw;
     Misc *misc = reinterpret_cast<Misc *>(smem + OFF_MISC);
     volatile int32_t *abort_flag = &misc->abort_flag;
 
@@ -190,22 +196,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(bar(&misc->full[i]), 1);
-            ptx::mbar_init(bar(&misc->empty[i]), 1);
+            ptx::mbar_init(bar(&misc->qk_full[i]), 1);
+            ptx::mbar_init(bar(&misc->qk_empty[i]), 1);
+            ptx::mbar_init(bar(&misc->pv_full[i]), 1);
+            ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
             ptx::mbar_init(bar(&misc->s_full[i]), 1);
-            ptx::mbar_init(bar(&misc->s_free[i]), 8);
             ptx::mbar_init(bar(&misc->p_ready[i]), 8);
             ptx::mbar_init(bar(&misc->pv_done[i]), 1);
         }
         ptx::mbar_init(bar(&misc->q_ready), 8);
         ptx::mbar_init(bar(&misc->o_free), 8);
-        ptx::mbar_init(bar(&misc->xbar[0]), 4);
-        ptx::mbar_init(bar(&misc->xbar[1]), 4);
-        ptx::mbar_init(bar(&misc->xlbar), 4);
         ptx::mbar_init(bar(&misc->drain), 1);
         misc->abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    for (int i = threadIdx.x; i < 3 * 128; i += blockDim.x)
+        (i < 256 ? misc->xtag[i >> 7][i & 127] : misc->xltag[i - 256]) = 0u;
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, 0);
@@ -252,128 +258,155 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
         walk.tile = walk.te = 0;   // idle partition
     }
 
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 6) {
+        // ------------------------------------------------------ TMA producers
+        // warp 0 fills the QK^T ring (own 32 tokens x 9 channel blocks), warp 6
+        // the P.V ring (64 tokens x this SM's 4 channel blocks). Completion of
+        // both CTAs' copies is counted on the leader's barriers.
+        const bool qk = (warp == 0);
         if (ptx::elect_one()) {
-            const uint32_t full0 = (rank == 0) ? bar(&misc->full[0]) : leader_bar(&misc->full[0]);
-            const uint32_t full1 = (rank == 0) ? bar(&misc->full[1]) : leader_bar(&misc->full[1]);
+            uint64_t *fullb = qk ? misc->qk_full : misc->pv_full;
+            uint64_t *emptyb = qk ? misc->qk_empty : misc->pv_empty;
+            const uint32_t tx = 2 * (qk ? STAGE_QK : STAGE_PV);
+            const uint32_t fb0 = (rank == 0) ? bar(&fullb[0]) : leader_bar(&fullb[0]);
+            const uint32_t fb1 = (rank == 0) ? bar(&fullb[1]) : leader_bar(&fullb[1]);
             int64_t k = 0;
             bool bad_page = false;
+            auto prefetch = [&](int32_t pg) {
+                if (pg < 0 || pg >= args.num_pages) return;
+                for (int j = 0; j < 8; ++j)
+                    ptx::tma_prefetch_3d(&map_ckv32, 64 * j, OWN * rank, pg);
+                ptx::tma_prefetch_3d(&map_kr32, 0, OWN * rank, pg);
+            };
             while (!*abort_flag && walk.next()) {
                 const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
+                if (qk)   // warm L2 for the first tiles of the segment
+                    for (int64_t t = walk.t_begin + 1; t < walk.t_begin + PREFETCH && t < walk.t_end; ++t)
+                        prefetch(trow[t]);
                 for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
                     const int s = static_cast<int>(k & 1);
                     int32_t page = trow[t];
                     if (page < 0 || page >= args.num_pages) { bad_page = true; page = 0; }
-                    if (t + 2 < walk.t_end) {  // warm L2 two tiles ahead (own rows)
-                        int32_t pg2 = trow[t + 2];
-                        if (pg2 >= 0 && pg2 < args.num_pages) {
-                            for (int j = 0; j < 8; ++j)
-                                ptx::tma_prefetch_3d(&map_ckv32, 64 * j, OWN * rank, pg2);
-                            ptx::tma_prefetch_3d(&map_kr32, 0, OWN * rank, pg2);
-                        }
-                    }
-                    if (k >= 2 && !wait_bounded(bar(&misc->empty[s]), ((k >> 1) - 1) & 1,
-                                                abort_flag, args.timeout_ns))
+                    if (qk && t + PREFETCH < walk.t_end) prefetch(trow[t + PREFETCH]);
+                    if (k >= 2 && !wait_bounded(bar(&emptyb[s]), ((k >> 1) - 1) & 1, abort_flag,
+                                                args.timeout_ns))
                         break;
-                    const uint32_t fb = s ? full1 : full0;
-                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(&misc->full[s]), 2 * TX_PER_CTA);
-                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
-                    for (int j = 0; j < 8; ++j)
-                        ptx::tma_load_3d_pair(st + j * (OWN * 128), &map_ckv32, fb, 64 * j,
-                                              OWN * rank, page);
-                    ptx::tma_load_3d_pair(st + 8 * (OWN * 128), &map_kr32, fb, 0, OWN * rank, page);
-                    for (int u = 0; u < 4; ++u) {
-                        const int blk = 4 * (u >> 1) + 2 * static_cast<int>(rank) + (u & 1);
-                        ptx::tma_load_3d_pair(st + STAGE_QK + u * (TOK * 128), &map_ckv64, fb,
-                                              64 * blk, 0, page);
+                    const uint32_t fb = s ? fb1 : fb0;
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(&fullb[s]), tx);
+                    if (qk) {
+                        const uint32_t st = base + OFF_QK + s * STAGE_QK;
+                        for (int j = 0; j < 8; ++j)
+                            ptx::tma_load_3d_pair(st + j * (OWN * 128), &map_ckv32, fb, 64 * j,
+                                                  OWN * rank, page);
+                        ptx::tma_load_3d_pair(st + 8 * (OWN * 128), &map_kr32, fb, 0, OWN * rank, page);
+                    } else {
+                        const uint32_t st = base + OFF_PV + s * STAGE_PV;
+                        for (int u = 0; u < 4; ++u) {
+                            const int blk = 4 * (u >> 1) + 2 * static_cast<int>(rank) + (u & 1);
+                            ptx::tma_load_3d_pair(st + u * (TOK * 128), &map_ckv64, fb, 64 * blk, 0,
+                                                  page);
+                        }
                     }
                 }
             }
             if (bad_page) record_error(kErrDeviceBounds);
-            // drain: the leader waits until every issued stage has landed
+            // drain: the leader waits until every issued slot has landed
             if (rank == 0) {
                 for (int64_t kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk)
-                    wait_bounded(bar(&misc->full[kk & 1]), (kk >> 1) & 1, abort_flag,
-                                 args.timeout_ns);
+                    wait_bounded(bar(&fullb[kk & 1]), (kk >> 1) & 1, abort_flag, args.timeout_ns);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer (leader)
+        // Two cursors: QK^T of tile kq and P.V of tile kp (kp < kq <= kp + 2,
+        // two score buffers). Whichever is ready is issued; the polls are
+        // non-blocking so a late KV tile never holds back a ready P.V.
         if (rank == 0 && ptx::elect_one()) {
-            int64_t k = 0;
-            int64_t g = 0;
-            bool ok = true;
-            auto issue_pv = [&](int64_t kp, bool first_of_seg) -> bool {
-                const int s = static_cast<int>(kp & 1);
-                if (!wait_bounded(bar(&misc->p_ready[s]), (kp >> 1) & 1, abort_flag, args.timeout_ns))
-                    return false;
-                ptx::tc_fence_after();
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES + STAGE_QK;
-                const uint32_t pbuf = base + OFF_P + s * P_BYTES;
-                for (int c = 0; c < 2; ++c) {
-                    for (int kk = 0; kk < TOK / 16; ++kk) {
-                        const uint64_t a = ptx::smem_desc(pbuf + kk * 32, 16, 1024, ptx::kSwizzle128B);
-                        const uint64_t b = ptx::smem_desc(st + (2 * c) * (TOK * 128) + kk * 2048,
-                                                          TOK * 128, 1024, ptx::kSwizzle128B);
-                        ptx::mma_bf16_ss<2>(tmem + TMEM_O + 128 * c, a, b, IDESC_PV,
-                                            (first_of_seg && kk == 0) ? 0u : 1u);
-                    }
-                }
-                ptx::mma_commit_pair(bar(&misc->empty[s]), 0x3);
-                ptx::mma_commit_pair(bar(&misc->pv_done[s]), 0x3);
-                return true;
-            };
-            while (ok && !*abort_flag && walk.next()) {
-                const int64_t k0 = k;
-                if (!wait_bounded(bar(&misc->q_ready), g & 1, abort_flag, args.timeout_ns)) break;
-                for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
-                    const int s = static_cast<int>(k & 1);
-                    if (!wait_bounded(bar(&misc->full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    if (k >= 2 && !wait_bounded(bar(&misc->s_free[s]), ((k >> 1) - 1) & 1,
-                                                abort_flag, args.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
-                    for (int j = 0; j < NB; ++j) {
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t a = ptx::smem_desc(base + OFF_Q + j * (ROWS_CTA * 128) + kk * 32,
-                                                              16, 1024, ptx::kSwizzle128B);
-                            const uint64_t b = ptx::smem_desc(st + j * (OWN * 128) + kk * 32, 16, 1024,
-                                                              ptx::kSwizzle128B);
-                            ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s, a, b, IDESC_QK,
-                                                (j | kk) ? 1u : 0u);
-                        }
-                    }
-                    ptx::mma_commit_pair(bar(&misc->s_full[s]), 0x3);
-                    if (k > k0) {
-                        if (k - 1 == k0 && g > 0) {
-                            if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag,
-                                              args.timeout_ns)) {
-                                ok = false;
-                                break;
+            SegmentWalker wq = walk, wp = walk;
+            bool q_has = wq.next(), p_has = wp.next();
+            int64_t tq = q_has ? wq.t_begin : 0, tp = p_has ? wp.t_begin : 0;
+            int64_t kq = 0, kp = 0, gq = 0, gp = 0;
+            bool q_ready_seen = false, o_free_seen = false;
+            uint64_t idle_since = ptx::globaltimer_ns();
+            uint32_t spins = 0;
+            while ((q_has || p_has) && !*abort_flag) {
+                bool progressed = false;
+                if (q_has && kq < kp + 2) {
+                    if (!q_ready_seen) q_ready_seen = ptx::mbar_test_wait(bar(&misc->q_ready), gq & 1);
+                    const int s = static_cast<int>(kq & 1);
+                    if (q_ready_seen && ptx::mbar_test_wait(bar(&misc->qk_full[s]), (kq >> 1) & 1)) {
+                        ptx::tc_fence_after();
+                        const uint32_t st = base + OFF_QK + s * STAGE_QK;
+                        for (int j = 0; j < NB; ++j) {
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t a = ptx::smem_desc(
+                                    base + OFF_Q + j * (ROWS_CTA * 128) + kk * 32, 16, 1024,
+                                    ptx::kSwizzle128B);
+                                const uint64_t b = ptx::smem_desc(st + j * (OWN * 128) + kk * 32, 16,
+                                                                  1024, ptx::kSwizzle128B);
+                                ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s, a, b, IDESC_QK,
+                                                    (j | kk) ? 1u : 0u);
                             }
                         }
-                        if (!issue_pv(k - 1, k - 1 == k0)) { ok = false; break; }
+                        ptx::mma_commit_pair(bar(&misc->qk_empty[s]), 0x3);
+                        ptx::mma_commit_pair(bar(&misc->s_full[s]), 0x3);
+                        ++kq;
+                        if (++tq == wq.t_end) {
+                            q_has = wq.next();
+                            ++gq;
+                            q_ready_seen = false;
+                            if (q_has) tq = wq.t_begin;
+                        }
+                        progressed = true;
                     }
                 }
-                if (!ok) break;
-                // value product of the segment's last tile
-                if (k - 1 == k0 && g > 0) {
-                    if (!wait_bounded(bar(&misc->o_free), (g - 1) & 1, abort_flag, args.timeout_ns))
-                        break;
+                if (p_has && kp < kq) {
+                    const bool first = (tp == wp.t_begin);
+                    if (first && gp > 0 && !o_free_seen)
+                        o_free_seen = ptx::mbar_test_wait(bar(&misc->o_free), (gp - 1) & 1);
+                    const int s = static_cast<int>(kp & 1);
+                    if ((!first || gp == 0 || o_free_seen) &&
+                        ptx::mbar_test_wait(bar(&misc->pv_full[s]), (kp >> 1) & 1) &&
+                        ptx::mbar_test_wait(bar(&misc->p_ready[s]), (kp >> 1) & 1)) {
+                        ptx::tc_fence_after();
+                        const uint32_t st = base + OFF_PV + s * STAGE_PV;
+                        const uint32_t pbuf = base + OFF_P + s * P_BYTES;
+                        for (int c = 0; c < 2; ++c) {
+                            for (int kk = 0; kk < TOK / 16; ++kk) {
+                                const uint64_t a =
+                                    ptx::smem_desc(pbuf + kk * 32, 16, 1024, ptx::kSwizzle128B);
+                                const uint64_t b = ptx::smem_desc(st + (2 * c) * (TOK * 128) + kk * 2048,
+                                                                  TOK * 128, 1024, ptx::kSwizzle128B);
+                                ptx::mma_bf16_ss<2>(tmem + TMEM_O + 128 * c, a, b, IDESC_PV,
+                                                    (first && kk == 0) ? 0u : 1u);
+                            }
+                        }
+                        ptx::mma_commit_pair(bar(&misc->pv_empty[s]), 0x3);
+                        ptx::mma_commit_pair(bar(&misc->pv_done[s]), 0x3);
+                        ++kp;
+                        if (++tp == wp.t_end) {
+                            p_has = wp.next();
+                            ++gp;
+                            o_free_seen = false;
+                            if (p_has) tp = wp.t_begin;
+                        }
+                        progressed = true;
+                    }
                 }
-                if (!issue_pv(k - 1, k - 1 == k0)) break;
-                ++g;
+                if (progressed) {
+                    spins = 0;
+                } else if ((++spins & 63u) == 0u) {
+                    const uint64_t now = ptx::globaltimer_ns();
+                    if (spins == 64u) idle_since = now;
+                    else if (static_cast<int64_t>(now - idle_since) > args.timeout_ns) {
+                        record_error(kErrTimeout);
+                        *abort_flag = 1;
+                    }
+                }
             }
             // every MMA issued so far has finished before tensor memory is freed
             ptx::mma_commit_pair(bar(&misc->drain), 0x1);
-            wait_bounded(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
+            wait_bounded<false>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
         }
     } else {
         // ------------------------------------------------------ softmax / epilogue
@@ -424,7 +457,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
             bool ok = true;
             for (int64_t t = t_begin; t < t_end; ++t, ++k) {
                 const int s = static_cast<int>(k & 1);
-                if (!wait_bounded(bar(&misc->s_full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                if (!wait_bounded<false>(bar(&misc->s_full[s]), (k >> 1) & 1, abort_flag,
+                                         args.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -432,8 +466,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
                 uint32_t sr[32];
                 ptx::tmem_ld32(tmem + lane_base + TMEM_S + 32 * s, sr);
                 ptx::tmem_wait_ld();
-                ptx::tc_fence_before();
-                arrive_leader(&misc->s_free[s]);
 
                 const int32_t tok0 = static_cast<int32_t>(t) * TOK + half * OWN;
                 float v[32];
@@ -443,14 +475,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
                     v[j] = (tok0 + j < vis) ? __uint_as_float(sr[j]) : -INFINITY;
                     mx = fmaxf(mx, v[j]);
                 }
-                misc->xmax[s][lt] = mx;
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(&misc->xbar[s]));
-                if (!wait_bounded(bar(&misc->xbar[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                // half-row maxima meet through tagged words: low 8 mantissa bits
+                // carry the tile tag, both lanes use the same truncated values
+                const uint32_t tag = static_cast<uint32_t>((k >> 1) % 255) + 1u;
+                const uint32_t mine = (__float_as_uint(mx) & 0xFFFFFF00u) | tag;
+                reinterpret_cast<volatile uint32_t *>(misc->xtag[s])[lt] = mine;
+                uint32_t other = 0;
+                if (!wait_word(&misc->xtag[s][lt ^ 64], tag, abort_flag, args.timeout_ns, &other)) {
                     ok = false;
                     break;
                 }
-                mx = fmaxf(mx, misc->xmax[s][lt ^ 64]);
+                mx = fmaxf(__uint_as_float(mine & 0xFFFFFF00u), __uint_as_float(other & 0xFFFFFF00u));
 
                 float alpha = 1.f;
                 if (mx > -INFINITY && (m_run == -INFINITY ||
@@ -471,8 +506,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
                 const bool need = (k > k0) && (alpha != 1.f);
                 if (__any_sync(0xffffffffu, need)) {
                     const int64_t kp = k - 1;
-                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
-                                      args.timeout_ns)) {
+                    if (!wait_bounded<false>(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                             args.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -492,8 +527,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
                 // P buffer s is free once the value product of tile k-2 is done
                 if (k >= 2) {
                     const int64_t kp = k - 2;
-                    if (!wait_bounded(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
-                                      args.timeout_ns)) {
+                    if (!wait_bounded<false>(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
+                                             args.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -519,16 +554,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeThreads, 1)
 
             // epilogue of this segment
             const int64_t kl = k - 1;
-            if (!wait_bounded(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
-                              args.timeout_ns))
+            if (!wait_bounded<false>(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
+                                     args.timeout_ns))
                 break;
             ptx::tc_fence_after();
-            misc->xl[lt] = l_run;
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(&misc->xlbar));
-            if (!wait_bounded(bar(&misc->xlbar), seg_no & 1, abort_flag, args.timeout_ns)) break;
+            const uint32_t ltag = static_cast<uint32_t>(seg_no % 255) + 1u;
             ++seg_no;
-            const float l_row = l_run + misc->xl[lt ^ 64];
+            const uint32_t lmine = (__float_as_uint(l_run) & 0xFFFFFF00u) | ltag;
+            reinterpret_cast<volatile uint32_t *>(misc->xltag)[lt] = lmine;
+            uint32_t lother = 0;
+            if (!wait_word(&misc->xltag[lt ^ 64], ltag, abort_flag, args.timeout_ns, &lother)) break;
+            // identical in both lanes: the same two truncated terms, added commutatively
+            const float l_row = __uint_as_float(lmine & 0xFFFFFF00u) + __uint_as_float(lother & 0xFFFFFF00u);
             const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
             float *dst = args.o_part + (slot * args.rows + grow) * DC;
 #pragma unroll 1
@@ -585,7 +622,7 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_STAGE = 20480;                     // Q rounded up to 1 KB multiple
 constexpr uint32_t OFF_P = OFF_STAGE + STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + pair::MISC_BYTES + 1024;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + pair::MISC_BYTES + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                            // 64 columns
 constexpr uint32_t TMEM_S = 128;                          // two 128-column score buffers

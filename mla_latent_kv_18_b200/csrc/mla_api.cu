@@ -78,8 +78,8 @@ mla_status device_ready() {
             cudaFuncSetAttribute(mla::decode_single_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::single::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::head_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 mla::kProjTok * 512 * 4) != cudaSuccess) {
+            cudaFuncSetAttribute(mla::proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::proj_smem_bytes(256)) != cudaSuccess) {
             st.status = MLA_ERR_CUDA;
             return;
         }
@@ -125,16 +125,59 @@ mla_status pool_map(CUtensorMap *m, const mla_pool *pool, int32_t channels, int3
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
 }
 
+mla_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// 3-D bf16 map with 128-byte swizzle: dims (d0 inner, d1, d2), byte strides s1, s2.
+mla_status map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {s1, s2};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
+}
+
+// out[t, h, :n_cols] = x[t, h, :K] W[h] on tensor cores (+ RoPE copy when rope != null).
+mla_status launch_proj(const void *x, const void *w, void *out, const void *rope, int32_t T,
+                       int32_t H, int32_t K, int32_t n_cols, int32_t out_stride, int32_t d_rope,
+                       cudaStream_t s) {
+    const int NT = T >= 256 ? 256 : ((T + 15) / 16) * 16;
+    CUtensorMap mw, mx;
+    mla_status st;
+    if ((st = map_3d(&mw, w, n_cols, K, H, uint64_t(n_cols) * 2, uint64_t(K) * n_cols * 2, 64, 64,
+                     1)) != MLA_OK)
+        return st;
+    if ((st = map_3d(&mx, x, K, H, T, uint64_t(K) * 2, uint64_t(H) * K * 2, 64, 1, NT)) != MLA_OK)
+        return st;
+    mla::ProjArgs a;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.rope = static_cast<const __nv_bfloat16 *>(rope);
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.T = T;
+    a.H = H;
+    a.K = K;
+    a.n_cols = n_cols;
+    a.out_stride = out_stride;
+    a.d_rope = d_rope;
+    a.NT = NT;
+    dim3 grid(H, (n_cols + 127) / 128, (T + NT - 1) / NT);
+    mla::proj_tc_kernel<<<grid, 128, mla::proj_smem_bytes(NT), s>>>(mw, mx, a);
+    return launch_status();
+}
+
 mla_status check_pool(const mla_pool *p, int32_t channels) {
     if (!p || !p->base) return MLA_ERR_INVALID_ARG;
     if (!aligned(p->base, 16)) return MLA_ERR_INVALID_ARG;
     if (p->token_stride < channels || p->page_stride < p->token_stride) return MLA_ERR_INVALID_ARG;
     if ((p->token_stride % 8) || (p->page_stride % 8)) return MLA_ERR_INVALID_ARG;
     return MLA_OK;
-}
-
-mla_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -209,26 +252,15 @@ mla_status mla_absorb_q(const mla_dims *dims, const void *q_c, const void *q_r, 
     mla_status st = check_dims(dims, false);
     if (st != MLA_OK) return st;
     if (num_tokens < 0) return MLA_ERR_INVALID_ARG;
-    if (dims->d_nope > 512) return MLA_ERR_UNSUPPORTED;
+    if (dims->d_nope > 4096 || dims->d_latent > 4096) return MLA_ERR_UNSUPPORTED;
     if (num_tokens == 0) return MLA_OK;
     if (!q_c || !q_r || !w_uk || !q_out) return MLA_ERR_INVALID_ARG;
     if (!aligned(q_c, 16) || !aligned(q_r, 16) || !aligned(w_uk, 16) || !aligned(q_out, 16))
         return MLA_ERR_INVALID_ARG;
     if ((st = device_ready()) != MLA_OK) return st;
-    mla::ProjArgs a;
-    a.x = static_cast<const __nv_bfloat16 *>(q_c);
-    a.w = static_cast<const __nv_bfloat16 *>(w_uk);
-    a.out = static_cast<__nv_bfloat16 *>(q_out);
-    a.rope = static_cast<const __nv_bfloat16 *>(q_r);
-    a.T = num_tokens;
-    a.H = dims->num_heads;
-    a.K = dims->d_nope;
-    a.n_cols = dims->d_latent;
-    a.out_stride = dims->d_latent + dims->d_rope;
-    a.d_rope = dims->d_rope;
-    dim3 grid(dims->num_heads, (dims->d_latent + 127) / 128, (num_tokens + mla::kProjTok - 1) / mla::kProjTok);
-    mla::head_proj_kernel<<<grid, 128, mla::kProjTok * a.K * 4, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_status();
+    return launch_proj(q_c, w_uk, q_out, q_r, num_tokens, dims->num_heads, dims->d_nope,
+                       dims->d_latent, dims->d_latent + dims->d_rope, dims->d_rope,
+                       static_cast<cudaStream_t>(stream));
 }
 
 mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w_uv, void *out,
@@ -236,25 +268,13 @@ mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w
     mla_status st = check_dims(dims, false);
     if (st != MLA_OK) return st;
     if (num_tokens < 0) return MLA_ERR_INVALID_ARG;
-    if (dims->d_latent > 512) return MLA_ERR_UNSUPPORTED;
+    if (dims->d_latent > 4096 || dims->d_v > 4096) return MLA_ERR_UNSUPPORTED;
     if (num_tokens == 0) return MLA_OK;
     if (!o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
     if (!aligned(o_lat, 16) || !aligned(w_uv, 16) || !aligned(out, 16)) return MLA_ERR_INVALID_ARG;
     if ((st = device_ready()) != MLA_OK) return st;
-    mla::ProjArgs a;
-    a.x = static_cast<const __nv_bfloat16 *>(o_lat);
-    a.w = static_cast<const __nv_bfloat16 *>(w_uv);
-    a.out = static_cast<__nv_bfloat16 *>(out);
-    a.rope = nullptr;
-    a.T = num_tokens;
-    a.H = dims->num_heads;
-    a.K = dims->d_latent;
-    a.n_cols = dims->d_v;
-    a.out_stride = dims->d_v;
-    a.d_rope = 0;
-    dim3 grid(dims->num_heads, (dims->d_v + 127) / 128, (num_tokens + mla::kProjTok - 1) / mla::kProjTok);
-    mla::head_proj_kernel<<<grid, 128, mla::kProjTok * a.K * 4, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_status();
+    return launch_proj(o_lat, w_uv, out, nullptr, num_tokens, dims->num_heads, dims->d_latent,
+                       dims->d_v, dims->d_v, 0, static_cast<cudaStream_t>(stream));
 }
 
 mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_pool *ckv,
@@ -308,7 +328,7 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
         if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
             return st;
-        mla::decode_pair_kernel<<<2 * num_parts, mla::kDecodeThreads, mla::pair::SMEM_BYTES, s>>>(
+        mla::decode_pair_kernel<<<2 * num_parts, mla::kPairThreads, mla::pair::SMEM_BYTES, s>>>(
             m32, m64, mkr, a);
     } else {
         CUtensorMap mc, mkr;

@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace mla {
@@ -116,47 +118,130 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-head projections on CUDA cores: out[t, h, col] = sum_k x[t, h, k] W[h, k, col].
-// grid (H, ceil(n_cols / 128), ceil(T / 32)), 128 threads, one output column
-// per thread and 32 tokens per block; x rows staged in shared memory as fp32.
-// For absorb-in (copy_rope) the block with blockIdx.y == 0 also copies q_r.
+// Per-head projections on tensor cores: out[t, h, col] = sum_k x[t, h, k] W[h, k, col]
+// (absorb-in: x = q_c, W = W_UK; absorb-out: x = o_lat, W = W_UV).
+// Swap-AB so the tiny token count is the MMA N: D[col, t] = W[h]^T[col, k] x^T[k, t],
+// M = 128 output columns per CTA, N = NT tokens (<= 256), K in 64-wide blocks.
+// W tiles are read MN-major (columns contiguous) and x tiles K-major, both by
+// TMA with 128-byte swizzle; out-of-range rows/columns are zero-filled by TMA.
+// grid (H, ceil(n_cols / 128), ceil(T / NT)), 128 threads: warp 0 streams the
+// K blocks through a 4-stage ring, one thread of warp 1 issues the MMAs, all
+// four warps drain TMEM (lane = output column) and store bf16.
 // ---------------------------------------------------------------------------
 struct ProjArgs {
-    const __nv_bfloat16 *x;      // [T, H, K]
-    const __nv_bfloat16 *w;      // [H, K, n_cols]
     __nv_bfloat16 *out;          // [T, H, out_stride]
-    const __nv_bfloat16 *rope;   // [T, H, d_rope] or null
-    int32_t T, H, K, n_cols, out_stride, d_rope;
+    const __nv_bfloat16 *rope;   // [T, H, d_rope] or null (absorb-in copies q_r)
+    int64_t timeout_ns;
+    int32_t T, H, K, n_cols, out_stride, d_rope, NT;
 };
 
-constexpr int kProjTok = 32;
+constexpr int kProjStages = 4;
+constexpr uint32_t kProjW = 2 * 64 * 128;   // two 64-column atoms x 64 K rows
 
-__global__ void __launch_bounds__(128) head_proj_kernel(const ProjArgs a) {
-    extern __shared__ float xs[];  // [kProjTok][K]
-    const int h = blockIdx.x;
-    const int col = blockIdx.y * 128 + threadIdx.x;
-    const int t0 = blockIdx.z * kProjTok;
-    const int nt = min(kProjTok, a.T - t0);
-    for (int i = threadIdx.x; i < nt * a.K; i += 128) {
-        const int t = i / a.K, k = i - t * a.K;
-        xs[t * a.K + k] = __bfloat162float(a.x[(static_cast<int64_t>(t0 + t) * a.H + h) * a.K + k]);
-    }
-    __syncthreads();
-    if (col < a.n_cols) {
-        float acc[kProjTok];
-#pragma unroll
-        for (int t = 0; t < kProjTok; ++t) acc[t] = 0.f;
-        const __nv_bfloat16 *wp = a.w + static_cast<int64_t>(h) * a.K * a.n_cols + col;
-        for (int k = 0; k < a.K; ++k) {
-            const float wv = __bfloat162float(wp[static_cast<int64_t>(k) * a.n_cols]);
-#pragma unroll
-            for (int t = 0; t < kProjTok; ++t) acc[t] = fmaf(xs[t * a.K + k], wv, acc[t]);
+__host__ __device__ constexpr uint32_t proj_stage_bytes(int NT) {
+    return kProjW + static_cast<uint32_t>(NT) * 128;
+}
+__host__ __device__ constexpr uint32_t proj_smem_bytes(int NT) {
+    return kProjStages * proj_stage_bytes(NT) + 1024 /* barriers */ + 1024 /* alignment */;
+}
+
+__global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CUtensorMap map_w,
+                                                      const __grid_constant__ CUtensorMap map_x,
+                                                      const ProjArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_base);
+    const uint32_t stage_bytes = proj_stage_bytes(a.NT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kProjStages * stage_bytes);
+    uint64_t *full = bars, *empty = bars + kProjStages, *done = bars + 2 * kProjStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kProjStages + 1);
+    int32_t *abort_flag = reinterpret_cast<int32_t *>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x, m0 = blockIdx.y * 128, t0 = blockIdx.z * a.NT;
+    const int nkb = (a.K + 63) / 64;
+    uint32_t tcols = 32;
+    while (tcols < static_cast<uint32_t>(a.NT)) tcols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kProjStages; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
         }
+        ptx::mbar_init(ptx::smem_u32(done), 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
+        ptx::tmem_relinquish<1>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int32_t *abort_v = abort_flag;
+
+    if (warp == 0) {
+        if (ptx::elect_one()) {
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = kb % kProjStages;
+                if (kb >= kProjStages &&
+                    !wait_bounded(ptx::smem_u32(&empty[s]), ((kb / kProjStages) - 1) & 1, abort_v,
+                                  a.timeout_ns))
+                    break;
+                const uint32_t st = base + s * stage_bytes;
+                const uint32_t fb = ptx::smem_u32(&full[s]);
+                ptx::mbar_arrive_expect_tx(fb, stage_bytes);
+                ptx::tma_load_3d(st, &map_w, fb, m0, kb * 64, h);
+                ptx::tma_load_3d(st + 64 * 128, &map_w, fb, m0 + 64, kb * 64, h);
+                ptx::tma_load_3d(st + kProjW, &map_x, fb, kb * 64, h, t0);
+            }
+            for (int k2 = (kb > kProjStages ? kb - kProjStages : 0); k2 < kb; ++k2)
+                wait_bounded(ptx::smem_u32(&full[k2 % kProjStages]), (k2 / kProjStages) & 1, abort_v,
+                             a.timeout_ns);
+        }
+    } else if (warp == 1) {
+        if (ptx::elect_one()) {
+            const uint32_t idesc = ptx::idesc_bf16(128, a.NT, 1, 0);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kProjStages;
+                if (!wait_bounded(ptx::smem_u32(&full[s]), (kb / kProjStages) & 1, abort_v,
+                                  a.timeout_ns))
+                    break;
+                ptx::tc_fence_after();
+                const uint32_t st = base + s * stage_bytes;
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = ptx::smem_desc(st + kk * 2048, 64 * 128, 1024, ptx::kSwizzle128B);
+                    const uint64_t bd = ptx::smem_desc(st + kProjW + kk * 32, 16, 1024, ptx::kSwizzle128B);
+                    ptx::mma_bf16_ss<1>(tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+                }
+                ptx::mma_commit(ptx::smem_u32(&empty[s]));
+            }
+            ptx::mma_commit(ptx::smem_u32(done));
+        }
+    }
+    // epilogue: TMEM lane = output column m0 + 32*warp + lane, column = token
+    const bool ok = wait_bounded(ptx::smem_u32(done), 0, abort_v, a.timeout_ns);
+    ptx::tc_fence_after();
+    const int col = m0 + 32 * warp + lane;
+    const int nt = min(a.NT, a.T - t0);
+    if (ok) {
+        for (int c0 = 0; c0 < a.NT; c0 += 32) {
+            uint32_t v[32];
+            ptx::tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, v);
+            ptx::tmem_wait_ld();
+            if (col < a.n_cols) {
 #pragma unroll
-        for (int t = 0; t < kProjTok; ++t)
-            if (t < nt)
-                a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + col] =
-                    __float2bfloat16_rn(acc[t]);
+                for (int j = 0; j < 32; ++j) {
+                    const int t = c0 + j;
+                    if (t < nt)
+                        a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + col] =
+                            __float2bfloat16_rn(__uint_as_float(v[j]));
+                }
+            }
+        }
     }
     if (a.rope && blockIdx.y == 0) {
         for (int i = threadIdx.x; i < nt * a.d_rope; i += 128) {
@@ -165,6 +250,10 @@ __global__ void __launch_bounds__(128) head_proj_kernel(const ProjArgs a) {
                 a.rope[(static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + j];
         }
     }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc<1>(tmem, tcols);
 }
 
 // One block waits on a barrier nothing completes; the bounded wait runs out
