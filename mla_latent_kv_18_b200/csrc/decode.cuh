@@ -336,15 +336,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const int s = static_cast<int>(kq & 1);
                     if (q_ready_seen && ptx::mbar_test_wait(bar(&misc->qk_full[s]), (kq >> 1) & 1)) {
                         ptx::tc_fence_after();
-                        const uint32_t st = base + OFF_QK + s * STAGE_QK;
+                        // descriptors advance by (byte offset >> 4) in the start-address field
+                        const uint64_t a0 = ptx::smem_desc(base + OFF_Q, 16, 1024, ptx::kSwizzle128B);
+                        const uint64_t b0 = ptx::smem_desc(base + OFF_QK + s * STAGE_QK, 16, 1024,
+                                                           ptx::kSwizzle128B);
+#pragma unroll
                         for (int j = 0; j < NB; ++j) {
+#pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
-                                const uint64_t a = ptx::smem_desc(
-                                    base + OFF_Q + j * (ROWS_CTA * 128) + kk * 32, 16, 1024,
-                                    ptx::kSwizzle128B);
-                                const uint64_t b = ptx::smem_desc(st + j * (OWN * 128) + kk * 32, 16,
-                                                                  1024, ptx::kSwizzle128B);
-                                ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s, a, b, IDESC_QK,
+                                ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s,
+                                                    a0 + ((j * (ROWS_CTA * 128) + kk * 32) >> 4),
+                                                    b0 + ((j * (OWN * 128) + kk * 32) >> 4), IDESC_QK,
                                                     (j | kk) ? 1u : 0u);
                             }
                         }
@@ -369,16 +371,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         ptx::mbar_test_wait(bar(&misc->pv_full[s]), (kp >> 1) & 1) &&
                         ptx::mbar_test_wait(bar(&misc->p_ready[s]), (kp >> 1) & 1)) {
                         ptx::tc_fence_after();
-                        const uint32_t st = base + OFF_PV + s * STAGE_PV;
-                        const uint32_t pbuf = base + OFF_P + s * P_BYTES;
+                        const uint64_t a0 = ptx::smem_desc(base + OFF_P + s * P_BYTES, 16, 1024,
+                                                           ptx::kSwizzle128B);
+                        const uint64_t b0 = ptx::smem_desc(base + OFF_PV + s * STAGE_PV, TOK * 128,
+                                                           1024, ptx::kSwizzle128B);
+#pragma unroll
                         for (int c = 0; c < 2; ++c) {
+#pragma unroll
                             for (int kk = 0; kk < TOK / 16; ++kk) {
-                                const uint64_t a =
-                                    ptx::smem_desc(pbuf + kk * 32, 16, 1024, ptx::kSwizzle128B);
-                                const uint64_t b = ptx::smem_desc(st + (2 * c) * (TOK * 128) + kk * 2048,
-                                                                  TOK * 128, 1024, ptx::kSwizzle128B);
-                                ptx::mma_bf16_ss<2>(tmem + TMEM_O + 128 * c, a, b, IDESC_PV,
-                                                    (first && kk == 0) ? 0u : 1u);
+                                ptx::mma_bf16_ss<2>(tmem + TMEM_O + 128 * c, a0 + ((kk * 32) >> 4),
+                                                    b0 + (((2 * c) * (TOK * 128) + kk * 2048) >> 4),
+                                                    IDESC_PV, (first && kk == 0) ? 0u : 1u);
                             }
                         }
                         ptx::mma_commit_pair(bar(&misc->pv_empty[s]), 0x3);
@@ -494,17 +497,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     m_run = mx;
                 }
                 const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
-                float psum = 0.f;
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     v[j] = exp2f(fmaf(v[j], args.scale_log2, -mb));   // -inf -> 0
-                    psum += v[j];
+                    ps[j & 3] += v[j];
                 }
-                l_run = fmaf(l_run, alpha, psum);
+                l_run = fmaf(l_run, alpha, (ps[0] + ps[1]) + (ps[2] + ps[3]));
 
                 // rescale the accumulated O rows held by this lane
                 const bool need = (k > k0) && (alpha != 1.f);
-                if (__any_sync(0xffffffffu, need)) {
+                const bool any_need = __any_sync(0xffffffffu, need);
+                if (any_need) {
                     const int64_t kp = k - 1;
                     if (!wait_bounded<false>(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
                                              args.timeout_ns)) {
@@ -524,15 +528,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                     ptx::tmem_wait_st();
                 }
-                // P buffer s is free once the value product of tile k-2 is done
-                if (k >= 2) {
-                    const int64_t kp = k - 2;
-                    if (!wait_bounded<false>(bar(&misc->pv_done[kp & 1]), (kp >> 1) & 1, abort_flag,
-                                             args.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                }
+                // P buffer s is free: the value product of tile k-2 was issued
+                // before QK^T of tile k (score-buffer rule) and MMAs retire in
+                // issue order, so it finished before s_full(k) arrived.
                 const uint32_t pb = base + OFF_P + s * P_BYTES;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -543,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                  pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
                 }
                 ptx::fence_proxy_async_smem();
-                ptx::tc_fence_before();
+                if (any_need) ptx::tc_fence_before();   // order the O rescale stores
                 arrive_leader(&misc->p_ready[s]);
             }
             if (!ok) break;
