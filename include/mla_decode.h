@@ -182,6 +182,34 @@ int64_t mla_decode_plan(const mla_dims *dims, const int32_t *seq_lens_host,
                         int32_t *part_first, int32_t *slot_count, int64_t *slot_base);
 
 /*
+ * Split-KV decode plus log-sum-exp combine (mla_decode_splitkv followed by
+ * mla_combine) that allocates nothing and needs no workspace from the caller.
+ * This entry point has no counterpart on the pages; it exists for callers that
+ * cannot hand out device memory at call time -- for example a plugin's enqueue
+ * routine inside an inference engine that owns the whole memory budget, or a
+ * latency-critical path where a cudaMalloc (and the device synchronisation it
+ * can imply) is not acceptable.
+ * The partial results live in a fixed scratch array of MLA_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) that the library keeps in device memory on every GPU where it is
+ * loaded, for the life of the process. Problems whose workspace
+ * (mla_decode_workspace_bytes) exceeds it are rejected with
+ * MLA_ERR_INVALID_ARG; nothing is launched then.
+ * The first call on a device looks up that device's copy of the array
+ * (cudaGetSymbolAddress), so make the first call on each device before any
+ * stream capture. All calls share the one array and it keeps whatever the last
+ * call left; every slot a call reads is written earlier by the same call, so
+ * nothing needs clearing, but calls whose kernels overlap on the GPU (different
+ * streams, no ordering between them) race on it and must be serialised by the
+ * caller. Arguments and outputs are those of mla_decode_splitkv and mla_combine.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const mla_pool *ckv,
+                                     const mla_pool *kr, int32_t num_pages,
+                                     const int32_t *block_table, int32_t max_pages_per_seq,
+                                     const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                                     void *o_lat, float *lse_out, void *stream);
+
+/*
  * Test hook for the bounded waits: launches one block that waits on a barrier
  * nothing will complete, with a limit of timeout_ns nanoseconds, after which it
  * records MLA_ERR_TIMEOUT in the device error word and returns. Lets a test

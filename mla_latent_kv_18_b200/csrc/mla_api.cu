@@ -387,6 +387,62 @@ mla_status mla_get_device_error(int32_t *code, void *stream) {
     return MLA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// Scratch for mla_decode_latent_noalloc: the partial results of the split-KV
+// step live here instead of in a caller workspace. One copy per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocState {
+    std::once_flag once;
+    void *ptr = nullptr;
+    mla_status status = MLA_OK;
+};
+NoallocState g_noalloc[kMaxDevices];
+
+// Device address of this device's scratch array, looked up once per device
+// with that device current.
+mla_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    NoallocState &st = g_noalloc[dev];
+    std::call_once(st.once, [&] {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            st.status = MLA_ERR_CUDA;
+        else
+            st.ptr = p;
+    });
+    *out = st.ptr;
+    return st.status;
+}
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const mla_pool *ckv,
+                                     const mla_pool *kr, int32_t num_pages,
+                                     const int32_t *block_table, int32_t max_pages_per_seq,
+                                     const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                                     void *o_lat, float *lse_out, void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    const size_t need = mla_decode_workspace_bytes(dims, batch, num_parts);
+    if (need == 0 || need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != MLA_OK) return st;
+    st = mla_decode_splitkv(dims, q, ckv, kr, num_pages, block_table, max_pages_per_seq, seq_lens,
+                            batch, num_parts, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream);
+    if (st != MLA_OK) return st;
+    return mla_combine(dims, scratch, MLA_NOALLOC_SCRATCH_BYTES, seq_lens, max_pages_per_seq, batch,
+                       num_parts, o_lat, lse_out, stream);
+}
+
 mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream) {
     if (timeout_ns <= 0) return MLA_ERR_INVALID_ARG;
     mla_status st = device_ready();
