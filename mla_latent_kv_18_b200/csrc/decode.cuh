@@ -7,17 +7,19 @@
 //   O = P c_KV                                (value product stays in latent space)
 //   partial = O / l,  lse = m * scale + ln l
 //
-// Two kernels share the pipeline shape: warp 0 streams KV pages with TMA into
-// a two-stage shared-memory ring, one thread of warp 1 issues tcgen05 MMAs
-// into tensor memory, and warps 2..5 run the softmax, rescale O when the
-// running maximum grows by more than 2^8, write P, and write the partials.
+// Two kernels share the pipeline shape: TMA producer warps stream KV pages
+// into shared-memory rings, one thread of warp 1 issues tcgen05 MMAs into
+// tensor memory, and warps 2..5 run the softmax, rescale O when the running
+// maximum grows by more than 2^8, write P, and write the partials.
 //
 //  * decode_pair_kernel (d_c 512, d_R 64, page = tile = 64 tokens): a CTA pair
 //    on two SMs. The fp32 accumulator O[128 rows x 512] is exactly one SM's
 //    256 KB of tensor memory, so the pair splits it: cta_group::2 MMAs with
 //    M = 128 give each SM the O rows of its 64 query rows. QK^T splits the
 //    tile's 64 tokens (32 per SM); P.V splits the 512 latent columns (256 per
-//    SM, as two N = 256 MMAs). No MMA work is duplicated.
+//    SM, as two N = 256 MMAs). No MMA work is duplicated. Six of Q's nine
+//    64-channel blocks are the QK^T A operand straight from tensor memory,
+//    which leaves shared memory for a three-slot QK^T ring.
 //  * decode_single_kernel (d_c 64, d_R 8, tile = 128 tokens = 2 pages): one
 //    CTA, cta_group::1, M = 128 rows; the 8-wide RoPE key is padded to the
 //    16-wide MMA K step with a zero core-matrix column in shared memory.
@@ -130,25 +132,28 @@ constexpr int NB = D / 64;                    // 9 K-blocks of 64 channels
 constexpr int ROWS_CTA = 64;                  // query rows per SM
 constexpr int TOK = 64;                       // tokens per tile (one page)
 constexpr int OWN = 32;                       // tokens per SM in QK^T
-constexpr uint32_t Q_BYTES = NB * ROWS_CTA * 128;           // 73728
+constexpr int QT = 6;                         // Q channel blocks 0..5 live in tensor memory
+constexpr uint32_t Q_BYTES = (NB - QT) * ROWS_CTA * 128;    // 24576: Q blocks 6..8
 constexpr uint32_t STAGE_QK = NB * OWN * 128;               // 36864: own 32 tokens x 9 blocks
 constexpr uint32_t STAGE_PV = 4 * TOK * 128;                // 32768: 64 tokens x this SM's 4 blocks
-constexpr int STAGES = 2;                                   // slots in each of the two rings
+constexpr int QK_STAGES = 3;                                // QK^T ring depth
+constexpr int PV_STAGES = 2;                                // P.V ring depth
 constexpr uint32_t P_BYTES = ROWS_CTA * 128;                // 64 rows x 64 tokens bf16
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_QK = OFF_Q + Q_BYTES;                // QK^T ring
-constexpr uint32_t OFF_PV = OFF_QK + STAGES * STAGE_QK;     // P.V ring
-constexpr uint32_t OFF_P = OFF_PV + STAGES * STAGE_PV;
-constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 229376
-constexpr int PREFETCH = 4;                                 // L2 prefetch distance in tiles
+constexpr uint32_t OFF_PV = OFF_QK + QK_STAGES * STAGE_QK;  // P.V ring
+constexpr uint32_t OFF_P = OFF_PV + PV_STAGES * STAGE_PV;
+constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 217088
 constexpr uint32_t MISC_BYTES = 3072;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES;   // dynamic smem base is 1 KB aligned
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
 constexpr uint32_t TMEM_S = 256;               // two 32-column score buffers
+constexpr uint32_t TMEM_Q = 320;               // Q blocks 0..5: 32 columns each (two bf16 per column)
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, 256, 0, 1);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(TMEM_Q + QT * 32 <= TMEM_COLS, "tensor memory budget");
 static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 0 &&
                   (OFF_MISC % 1024) == 0, "align");
 }  // namespace pair
@@ -157,7 +162,8 @@ static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 
 struct Misc {
     uint64_t full[2], empty[2], s_full[2], s_free[2], p_ready[2], pv_done[2], q_ready, o_free;
     uint64_t drain;                   // MMA drain before tensor memory is freed
-    uint64_t qk_full[2], qk_empty[2], pv_full[2], pv_empty[2];   // the pair kernel's two rings
+    uint64_t qk_full[pair::QK_STAGES], qk_empty[pair::QK_STAGES];   // the pair kernel's two rings
+    uint64_t pv_full[pair::PV_STAGES], pv_empty[pair::PV_STAGES];
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t cur_b;
@@ -195,9 +201,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < QK_STAGES; ++i) {
             ptx::mbar_init(bar(&misc->qk_full[i]), 1);
             ptx::mbar_init(bar(&misc->qk_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(&misc->pv_full[i]), 1);
             ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
             ptx::mbar_init(bar(&misc->s_full[i]), 1);
@@ -267,32 +275,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (ptx::elect_one()) {
             uint64_t *fullb = qk ? misc->qk_full : misc->pv_full;
             uint64_t *emptyb = qk ? misc->qk_empty : misc->pv_empty;
+            const int nst = qk ? QK_STAGES : PV_STAGES;
             const uint32_t tx = 2 * (qk ? STAGE_QK : STAGE_PV);
-            const uint32_t fb0 = (rank == 0) ? bar(&fullb[0]) : leader_bar(&fullb[0]);
-            const uint32_t fb1 = (rank == 0) ? bar(&fullb[1]) : leader_bar(&fullb[1]);
             int64_t k = 0;
             bool bad_page = false;
-            auto prefetch = [&](int32_t pg) {
-                if (pg < 0 || pg >= args.num_pages) return;
-                for (int j = 0; j < 8; ++j)
-                    ptx::tma_prefetch_3d(&map_ckv32, 64 * j, OWN * rank, pg);
-                ptx::tma_prefetch_3d(&map_kr32, 0, OWN * rank, pg);
-            };
             while (!*abort_flag && walk.next()) {
                 const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
-                if (qk)   // warm L2 for the first tiles of the segment
-                    for (int64_t t = walk.t_begin + 1; t < walk.t_begin + PREFETCH && t < walk.t_end; ++t)
-                        prefetch(trow[t]);
                 for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
-                    const int s = static_cast<int>(k & 1);
+                    const int s = static_cast<int>(k % nst);
+                    const int64_t use = k / nst;
                     int32_t page = trow[t];
                     if (page < 0 || page >= args.num_pages) { bad_page = true; page = 0; }
-                    if (qk && t + PREFETCH < walk.t_end) prefetch(trow[t + PREFETCH]);
-                    if (k >= 2 && !wait_bounded(bar(&emptyb[s]), ((k >> 1) - 1) & 1, abort_flag,
-                                                args.timeout_ns))
+                    if (use >= 1 && !wait_bounded(bar(&emptyb[s]), (use - 1) & 1, abort_flag,
+                                                  args.timeout_ns))
                         break;
-                    const uint32_t fb = s ? fb1 : fb0;
-                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(&fullb[s]), tx);
+                    const uint32_t fb = (rank == 0) ? bar(&fullb[s]) : leader_bar(&fullb[s]);
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(fb, tx);
                     if (qk) {
                         const uint32_t st = base + OFF_QK + s * STAGE_QK;
                         for (int j = 0; j < 8; ++j)
@@ -312,8 +310,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (bad_page) record_error(kErrDeviceBounds);
             // drain: the leader waits until every issued slot has landed
             if (rank == 0) {
-                for (int64_t kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk)
-                    wait_bounded(bar(&fullb[kk & 1]), (kk >> 1) & 1, abort_flag, args.timeout_ns);
+                for (int64_t kk = (k >= nst ? k - nst : 0); kk < k; ++kk)
+                    wait_bounded(bar(&fullb[kk % nst]), (kk / nst) & 1, abort_flag, args.timeout_ns);
             }
         }
     } else if (warp == 1) {
@@ -333,25 +331,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 bool progressed = false;
                 if (q_has && kq < kp + 2) {
                     if (!q_ready_seen) q_ready_seen = ptx::mbar_test_wait(bar(&misc->q_ready), gq & 1);
-                    const int s = static_cast<int>(kq & 1);
-                    if (q_ready_seen && ptx::mbar_test_wait(bar(&misc->qk_full[s]), (kq >> 1) & 1)) {
+                    const int s = static_cast<int>(kq % QK_STAGES);
+                    const int sb = static_cast<int>(kq & 1);
+                    if (q_ready_seen &&
+                        ptx::mbar_test_wait(bar(&misc->qk_full[s]), (kq / QK_STAGES) & 1)) {
                         ptx::tc_fence_after();
                         // descriptors advance by (byte offset >> 4) in the start-address field
                         const uint64_t a0 = ptx::smem_desc(base + OFF_Q, 16, 1024, ptx::kSwizzle128B);
                         const uint64_t b0 = ptx::smem_desc(base + OFF_QK + s * STAGE_QK, 16, 1024,
                                                            ptx::kSwizzle128B);
+                        const uint32_t d = tmem + TMEM_S + 32 * sb;
 #pragma unroll
                         for (int j = 0; j < NB; ++j) {
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
-                                ptx::mma_bf16_ss<2>(tmem + TMEM_S + 32 * s,
-                                                    a0 + ((j * (ROWS_CTA * 128) + kk * 32) >> 4),
-                                                    b0 + ((j * (OWN * 128) + kk * 32) >> 4), IDESC_QK,
-                                                    (j | kk) ? 1u : 0u);
+                                const uint64_t b = b0 + ((j * (OWN * 128) + kk * 32) >> 4);
+                                const uint32_t acc = (j | kk) ? 1u : 0u;
+                                if (j < QT)   // A from tensor memory: 8 columns per 16-channel step
+                                    ptx::mma_bf16_ts<2>(d, tmem + TMEM_Q + 32 * j + 8 * kk, b, IDESC_QK,
+                                                        acc);
+                                else
+                                    ptx::mma_bf16_ss<2>(
+                                        d, a0 + (((j - QT) * (ROWS_CTA * 128) + kk * 32) >> 4), b,
+                                        IDESC_QK, acc);
                             }
                         }
                         ptx::mma_commit_pair(bar(&misc->qk_empty[s]), 0x3);
-                        ptx::mma_commit_pair(bar(&misc->s_full[s]), 0x3);
+                        ptx::mma_commit_pair(bar(&misc->s_full[sb]), 0x3);
                         ++kq;
                         if (++tq == wq.t_end) {
                             q_has = wq.next();
@@ -429,18 +435,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 else ptx::mbar_arrive_cluster(leader_bar(b));
             }
         };
+        // Q of sequence b: channel blocks 0..5 into tensor memory in the
+        // duplicated 2-SM A layout (this lane holds row lt % 64, so lanes lt and
+        // lt ^ 64 carry the same row), blocks 6..8 into shared memory
+        // (128-byte swizzled, K-major).
         auto load_q = [&](int32_t b) {
             const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
-            for (int idx = st_tid; idx < ROWS_CTA * (D / 8); idx += 128) {
-                const int r = idx / (D / 8);
-                const int cc = idx - r * (D / 8);
+            const __nv_bfloat16 *qrow = qb + static_cast<int64_t>(real_row ? grow : 0) * D;
+#pragma unroll 1
+            for (int j = 0; j < QT; ++j) {
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (real_row) v = ld_global_nc_v4(qrow + 64 * j + 8 * i);
+                    w[4 * i] = v.x;
+                    w[4 * i + 1] = v.y;
+                    w[4 * i + 2] = v.z;
+                    w[4 * i + 3] = v.w;
+                }
+                ptx::tmem_st32(tmem + lane_base + TMEM_Q + 32 * j, w);
+            }
+            for (int idx = st_tid; idx < ROWS_CTA * (NB - QT) * 8; idx += 128) {
+                const int r = idx / ((NB - QT) * 8);
+                const int cc = idx - r * ((NB - QT) * 8);   // 16-byte chunk among blocks 6..8
                 const int gr = ROWS_CTA * static_cast<int>(rank) + r;
                 uint4 v = make_uint4(0, 0, 0, 0);
-                if (gr < args.rows) v = ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + cc * 8);
+                if (gr < args.rows)
+                    v = ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + 64 * QT + cc * 8);
                 const uint32_t dst = base + OFF_Q + (cc >> 3) * (ROWS_CTA * 128) + sw128(r, cc & 7);
                 st_shared_v4(dst, v.x, v.y, v.z, v.w);
             }
+            ptx::tmem_wait_st();
             ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
             arrive_leader(&misc->q_ready);
         };
 
