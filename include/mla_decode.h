@@ -210,6 +210,27 @@ mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const 
                                      void *o_lat, float *lse_out, void *stream);
 
 /*
+ * Debug gather, the check on the page lookup of the decode calls: token t of
+ * sequence b is row t % 64 of page block_table[b][t / 64] of the pool
+ * ("MLA operator design" page §3, its 64-token pages). Uses the same TMA pool
+ * descriptor construction and table lookup as mla_decode_splitkv and writes
+ *   out[b, t, :] = pool[block_table[b][t / 64]][t % 64][0 : width]   (bit copy)
+ * for t < seq_lens[b]; rows t >= seq_lens[b] of out are left untouched.
+ * pool: base 16-byte aligned, strides in elements, multiples of 8, token
+ * stride >= width. width: 8..512, a multiple of 8, and of 64 when above 64.
+ * block_table [batch, max_pages_per_seq] int32, seq_lens [batch] int32 and
+ * out [batch, max_len, width] bf16 are device pointers owned by the caller.
+ * Returns MLA_ERR_INVALID_ARG on bad sizes or pointers (nothing launched);
+ * a page id outside [0, num_pages) or seq_lens[b] outside [0, max_len] (or
+ * beyond max_pages_per_seq pages) sets MLA_ERR_DEVICE_BOUNDS in the device
+ * error word. Table entries past a sequence's last page are never read.
+ */
+mla_status mla_debug_gather(const mla_pool *pool, int32_t width, int32_t num_pages,
+                            const int32_t *block_table, int32_t max_pages_per_seq,
+                            const int32_t *seq_lens, int32_t batch, int32_t max_len, void *out,
+                            void *stream);
+
+/*
  * Test hook for the bounded waits: launches one block that waits on a barrier
  * nothing will complete, with a limit of timeout_ns nanoseconds, after which it
  * records MLA_ERR_TIMEOUT in the device error word and returns. Lets a test

@@ -154,6 +154,23 @@ def get_device_error(stream=None):
     return code.value
 
 
+def debug_gather(pool, block_table, seq_lens, max_len, out=None, stream=None):
+    """Gathered rows of a [pages, 64, width] (possibly channel-sliced) pool:
+    out[b, t, :] = pool[block_table[b, t // 64], t % 64, :] for t < seq_lens[b]
+    (bf16 bit copy; other rows of out are left as they were, zeros if allocated
+    here). Uses the decode calls' page lookup and TMA pool descriptors."""
+    B, max_pages = block_table.shape
+    width = pool.shape[2]
+    if out is None:
+        out = torch.zeros((B, max_len, width), dtype=torch.bfloat16, device=pool.device)
+    p = _pool(pool)
+    _b.check(_b.lib.mla_debug_gather(ctypes.byref(p), width, pool.shape[0], _ptr(block_table),
+                                     max_pages, _ptr(seq_lens), B, max_len, _ptr(out),
+                                     _stream(stream)),
+             "mla_debug_gather")
+    return out
+
+
 def debug_wait_timeout(timeout_ns, stream=None):
     _b.check(_b.lib.mla_debug_wait_timeout(int(timeout_ns), _stream(stream)),
              "mla_debug_wait_timeout")

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include <cuda.h>
@@ -57,6 +58,8 @@ float scale_of(const mla_dims *d) {
                                   : static_cast<float>(1.0 / std::sqrt(double(d->d_nope + d->d_rope)));
 }
 
+constexpr int32_t kGatherMaxWidth = 512;
+
 // Per-device one-time state: capability check and kernel attributes.
 struct DeviceState {
     std::once_flag once;
@@ -79,7 +82,9 @@ mla_status device_ready() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::single::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 mla::proj_smem_bytes(256)) != cudaSuccess) {
+                                 mla::proj_smem_bytes(256)) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 64 * kGatherMaxWidth * 2) != cudaSuccess) {
             st.status = MLA_ERR_CUDA;
             return;
         }
@@ -167,8 +172,9 @@ mla_status launch_proj(const void *x, const void *w, void *out, const void *rope
     a.out_stride = out_stride;
     a.d_rope = d_rope;
     a.NT = NT;
+    a.stages = std::min(mla::kProjStages, (K + 63) / 64);
     dim3 grid(H, (n_cols + 127) / 128, (T + NT - 1) / NT);
-    mla::proj_tc_kernel<<<grid, 128, mla::proj_smem_bytes(NT), s>>>(mw, mx, a);
+    mla::proj_tc_kernel<<<grid, 128, mla::proj_smem_bytes(NT, a.stages), s>>>(mw, mx, a);
     return launch_status();
 }
 
@@ -441,6 +447,40 @@ mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const 
     if (st != MLA_OK) return st;
     return mla_combine(dims, scratch, MLA_NOALLOC_SCRATCH_BYTES, seq_lens, max_pages_per_seq, batch,
                        num_parts, o_lat, lse_out, stream);
+}
+
+mla_status mla_debug_gather(const mla_pool *pool, int32_t width, int32_t num_pages,
+                            const int32_t *block_table, int32_t max_pages_per_seq,
+                            const int32_t *seq_lens, int32_t batch, int32_t max_len, void *out,
+                            void *stream) {
+    if (width < 8 || width > kGatherMaxWidth || (width % 8) || (width > 64 && (width % 64)))
+        return MLA_ERR_INVALID_ARG;
+    if (num_pages <= 0 || max_pages_per_seq <= 0 || batch < 0 || max_len <= 0) return MLA_ERR_INVALID_ARG;
+    if (!block_table || !seq_lens || !out || !aligned(out, 16) || !aligned(block_table, 4) ||
+        !aligned(seq_lens, 4))
+        return MLA_ERR_INVALID_ARG;
+    mla_status st = check_pool(pool, width);
+    if (st != MLA_OK) return st;
+    if ((st = device_ready()) != MLA_OK) return st;
+    if (batch == 0) return MLA_OK;
+    const uint32_t box_ch = static_cast<uint32_t>(width < 64 ? width : 64);
+    CUtensorMap m;
+    if ((st = pool_map(&m, pool, width, num_pages, box_ch, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != MLA_OK)
+        return st;
+    mla::GatherArgs a;
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.batch = batch;
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    a.width = width;
+    a.box_ch = static_cast<int32_t>(box_ch);
+    a.max_len = max_len;
+    dim3 grid(batch, max_pages_per_seq);
+    mla::gather_kernel<<<grid, 128, 64 * width * 2, static_cast<cudaStream_t>(stream)>>>(m, a);
+    return launch_status();
 }
 
 mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream) {

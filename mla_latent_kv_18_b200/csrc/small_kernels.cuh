@@ -68,7 +68,8 @@ struct CombineArgs {
     int32_t batch, max_pages, n_q, rows, d_c, tile_tokens, num_parts;
 };
 
-// grid (batch, ceil(R / 4)), 128 threads: one warp per query row.
+// grid (batch, ceil(R / 4)), 128 threads: one warp per query row; each lane
+// keeps eight slots' loads in flight.
 __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
     __shared__ int64_t s_base, s_count;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -93,18 +94,34 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
     const float L = (m > -INFINITY) ? m + __logf(z) : -INFINITY;
 
     __nv_bfloat16 *dst = a.o_lat + (static_cast<int64_t>(b) * a.rows + r) * a.d_c;
+    const float *lse_r = a.lse_part + base * a.rows + r;
+    const float *o_r = a.o_part + (base * a.rows + r) * a.d_c;
+    const int64_t slot_stride = static_cast<int64_t>(a.rows) * a.d_c;
+    constexpr int U = 8;   // slots in flight per thread
     for (int c0 = 4 * lane; c0 < a.d_c; c0 += 128) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (m > -INFINITY) {
-            for (int64_t s = 0; s < cnt; ++s) {
-                const float ls = a.lse_part[(base + s) * a.rows + r];
-                const float w = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
-                const float4 v = *reinterpret_cast<const float4 *>(
-                    a.o_part + ((base + s) * a.rows + r) * a.d_c + c0);
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-                acc.z = fmaf(w, v.z, acc.z);
-                acc.w = fmaf(w, v.w, acc.w);
+            for (int64_t s0 = 0; s0 < cnt; s0 += U) {
+                float w[U];
+                float4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t s = s0 + u;
+                    w[u] = 0.f;
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (s < cnt) {
+                        const float ls = lse_r[s * a.rows];
+                        w[u] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
+                        v[u] = *reinterpret_cast<const float4 *>(o_r + s * slot_stride + c0);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    acc.x = fmaf(w[u], v[u].x, acc.x);
+                    acc.y = fmaf(w[u], v[u].y, acc.y);
+                    acc.z = fmaf(w[u], v[u].z, acc.z);
+                    acc.w = fmaf(w[u], v[u].w, acc.w);
+                }
             }
         }
         __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
@@ -133,6 +150,7 @@ struct ProjArgs {
     const __nv_bfloat16 *rope;   // [T, H, d_rope] or null (absorb-in copies q_r)
     int64_t timeout_ns;
     int32_t T, H, K, n_cols, out_stride, d_rope, NT;
+    int32_t stages;              // ring depth: min(kProjStages, K blocks)
 };
 
 constexpr int kProjStages = 4;
@@ -141,8 +159,8 @@ constexpr uint32_t kProjW = 2 * 64 * 128;   // two 64-column atoms x 64 K rows
 __host__ __device__ constexpr uint32_t proj_stage_bytes(int NT) {
     return kProjW + static_cast<uint32_t>(NT) * 128;
 }
-__host__ __device__ constexpr uint32_t proj_smem_bytes(int NT) {
-    return kProjStages * proj_stage_bytes(NT) + 1024 /* barriers */ + 1024 /* alignment */;
+__host__ __device__ constexpr uint32_t proj_smem_bytes(int NT, int stages = kProjStages) {
+    return static_cast<uint32_t>(stages) * proj_stage_bytes(NT) + 1024 /* barriers */ + 1024 /* alignment */;
 }
 
 __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CUtensorMap map_w,
@@ -153,9 +171,10 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_base);
     const uint32_t stage_bytes = proj_stage_bytes(a.NT);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kProjStages * stage_bytes);
-    uint64_t *full = bars, *empty = bars + kProjStages, *done = bars + 2 * kProjStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kProjStages + 1);
+    const int S = a.stages;   // ring depth, <= kProjStages
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * stage_bytes);
+    uint64_t *full = bars, *empty = bars + S, *done = bars + 2 * S;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
     int32_t *abort_flag = reinterpret_cast<int32_t *>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x, m0 = blockIdx.y * 128, t0 = blockIdx.z * a.NT;
@@ -164,7 +183,7 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
     while (tcols < static_cast<uint32_t>(a.NT)) tcols <<= 1;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kProjStages; ++i) {
+        for (int i = 0; i < S; ++i) {
             ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
             ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
         }
@@ -186,9 +205,9 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
         if (ptx::elect_one()) {
             int kb = 0;
             for (; kb < nkb; ++kb) {
-                const int s = kb % kProjStages;
-                if (kb >= kProjStages &&
-                    !wait_bounded(ptx::smem_u32(&empty[s]), ((kb / kProjStages) - 1) & 1, abort_v,
+                const int s = kb % S;
+                if (kb >= S &&
+                    !wait_bounded(ptx::smem_u32(&empty[s]), ((kb / S) - 1) & 1, abort_v,
                                   a.timeout_ns))
                     break;
                 const uint32_t st = base + s * stage_bytes;
@@ -198,16 +217,16 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
                 ptx::tma_load_3d(st + 64 * 128, &map_w, fb, m0 + 64, kb * 64, h);
                 ptx::tma_load_3d(st + kProjW, &map_x, fb, kb * 64, h, t0);
             }
-            for (int k2 = (kb > kProjStages ? kb - kProjStages : 0); k2 < kb; ++k2)
-                wait_bounded(ptx::smem_u32(&full[k2 % kProjStages]), (k2 / kProjStages) & 1, abort_v,
+            for (int k2 = (kb > S ? kb - S : 0); k2 < kb; ++k2)
+                wait_bounded(ptx::smem_u32(&full[k2 % S]), (k2 / S) & 1, abort_v,
                              a.timeout_ns);
         }
     } else if (warp == 1) {
         if (ptx::elect_one()) {
             const uint32_t idesc = ptx::idesc_bf16(128, a.NT, 1, 0);
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kProjStages;
-                if (!wait_bounded(ptx::smem_u32(&full[s]), (kb / kProjStages) & 1, abort_v,
+                const int s = kb % S;
+                if (!wait_bounded(ptx::smem_u32(&full[s]), (kb / S) & 1, abort_v,
                                   a.timeout_ns))
                     break;
                 ptx::tc_fence_after();
@@ -258,6 +277,64 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
 
 // One block waits on a barrier nothing completes; the bounded wait runs out
 // after timeout_ns and records kErrTimeout.
+// ---------------------------------------------------------------------------
+// Debug gather: the page lookup of the decode kernels (token t of sequence b
+// is row t % 64 of page block_table[b][t / 64], "MLA operator design" page §3)
+// through a TMA pool descriptor like theirs, written out densely.
+// grid (batch, max_pages), 128 threads, dynamic smem 64 x width x 2 bytes:
+// CTA (b, pg) loads page pg of sequence b as width / box_ch boxes of
+// [64 tokens x box_ch channels] and copies its valid tokens to out.
+// ---------------------------------------------------------------------------
+struct GatherArgs {
+    const int32_t *block_table;  // [B, max_pages]
+    const int32_t *seq_lens;     // [B]
+    __nv_bfloat16 *out;          // [B, max_len, width]
+    int64_t timeout_ns;
+    int32_t batch, max_pages, num_pages, width, box_ch, max_len;
+};
+
+__global__ void __launch_bounds__(128) gather_kernel(const __grid_constant__ CUtensorMap map,
+                                                     const GatherArgs a) {
+    extern __shared__ __align__(128) uint8_t gather_smem[];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int32_t abort_flag;
+    const int32_t b = blockIdx.x, pg = blockIdx.y;
+    const int32_t L = a.seq_lens[b];
+    if (L < 0 || L > a.max_len || static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * 64) {
+        if (threadIdx.x == 0 && pg == 0) record_error(kErrDeviceBounds);
+        return;
+    }
+    if (static_cast<int64_t>(pg) * 64 >= L) return;   // entries past the last page are not read
+    const int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_pages + pg];
+    if (page < 0 || page >= a.num_pages) {
+        if (threadIdx.x == 0) record_error(kErrDeviceBounds);
+        return;
+    }
+    const uint32_t base = ptx::smem_u32(gather_smem);
+    const uint32_t bb = ptx::smem_u32(&bar);
+    const int nbox = a.width / a.box_ch;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bb, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::mbar_arrive_expect_tx(bb, static_cast<uint32_t>(64 * a.width * 2));
+        for (int j = 0; j < nbox; ++j)
+            ptx::tma_load_3d(base + static_cast<uint32_t>(j * 64 * a.box_ch * 2), &map, bb,
+                             j * a.box_ch, 0, page);
+    }
+    __syncthreads();
+    if (!wait_bounded<false>(bb, 0, &abort_flag, a.timeout_ns)) return;
+    const int n = min(64, L - pg * 64);
+    const int c8n = a.width / 8;
+    __nv_bfloat16 *dst = a.out + (static_cast<int64_t>(b) * a.max_len + static_cast<int64_t>(pg) * 64) * a.width;
+    for (int idx = threadIdx.x; idx < n * c8n; idx += blockDim.x) {
+        const int t = idx / c8n, c = (idx - t * c8n) * 8;
+        const int j = c / a.box_ch, cin = c - j * a.box_ch;
+        const uint4 v = *reinterpret_cast<const uint4 *>(gather_smem + (static_cast<int64_t>(j) * 64 + t) * a.box_ch * 2 + cin * 2);
+        *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(t) * a.width + c) = v;
+    }
+}
+
 __global__ void wait_timeout_kernel(int64_t timeout_ns) {
     __shared__ __align__(8) uint64_t b;
     __shared__ int32_t abort_flag;

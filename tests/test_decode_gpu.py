@@ -236,6 +236,46 @@ def test_interleaved_pool_matches_separate_pools(api):
     assert torch.equal(r1["out"], r2["out"])
 
 
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("dsv3", dict(batch=3, heads=16, seq_len=300)),
+                                     ("ragged", dict(batch=6, heads=16, ragged=(1, 700))),
+                                     ("retrofit", dict(batch=3, seq_len=250))])
+def test_gather_is_bit_exact(api, name, kw):
+    """The decode calls' page lookup, written out densely through the same TMA
+    pool descriptors, equals the oracle's gather bit for bit: both pools,
+    every visible token, nothing written past a sequence's length."""
+    w = workload(name, **kw)
+    inp = make_inputs(w, seed=12)
+    d = to_device(inp, "cuda")
+    max_len = int(inp["seq_lens"].max()) + 5
+    for pool_name in ("ckv_pool", "kr_pool"):
+        got = api.debug_gather(d[pool_name], d["block_table"], d["seq_lens"], max_len)
+        assert api.get_device_error() == 0
+        ref = oracle.gather(inp[pool_name], inp["block_table"], inp["seq_lens"], 64, max_len)
+        assert np.array_equal(got.cpu().view(torch.int16).numpy().view(np.uint16), ref), pool_name
+
+
+def test_gather_from_interleaved_pool_is_bit_exact(api):
+    w = workload("dsv3", batch=3, heads=16, seq_len=300)
+    inp = make_inputs(w, seed=13)
+    both = torch.cat([inp["ckv_pool"], inp["kr_pool"]], dim=-1).cuda()   # [pages, 64, 576]
+    bt, sl = inp["block_table"].cuda(), inp["seq_lens"].cuda()
+    for view, pool_name in ((both[..., :512], "ckv_pool"), (both[..., 512:], "kr_pool")):
+        got = api.debug_gather(view, bt, sl, 300)
+        ref = oracle.gather(inp[pool_name], inp["block_table"], inp["seq_lens"], 64, 300)
+        assert np.array_equal(got.cpu().view(torch.int16).numpy().view(np.uint16), ref), pool_name
+    assert api.get_device_error() == 0
+
+
+def test_gather_bad_page_id_sets_device_error(api):
+    w = workload("dsv3", batch=2, heads=16, seq_len=300)
+    inp = make_inputs(w, seed=14)
+    d = to_device(inp, "cuda")
+    d["block_table"][1, 3] = -7
+    api.debug_gather(d["ckv_pool"], d["block_table"], d["seq_lens"], 300)
+    assert api.get_device_error() == 4
+    assert api.get_device_error() == 0
+
+
 def test_repeat_calls_are_bitwise_identical(api):
     w = workload("ragged", batch=8, heads=128, ragged=(500, 5000))
     inp_d = to_device(make_inputs(w, seed=9), "cuda")
