@@ -4,8 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long|dsv3|ragged|retrofit|tiny]
 
-A step is one pass of the whole decode path -- absorb-in, split-KV decode,
-log-sum-exp combine, absorb-out -- over one batch of the workload (default:
+A step is one pass of the whole decode path -- absorb-in, split-KV decode, and
+the log-sum-exp combine fused with absorb-out (mla_combine_absorb_out; with
+--unfused the two run as separate calls) -- over one batch of the workload (default:
 batch 16, 128 heads, 65536 cached tokens per sequence, d_c 512, d_R 64,
 page_size 64, shuffled page table). Inputs (1.2 GB of latent cache) exceed the
 126 MB L2, so no flush is needed between steps. With N GPUs each rank runs its
@@ -48,6 +49,8 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run combine and absorb-out as two calls instead of the fused one")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -257,9 +260,13 @@ def main():
                            dims, dec.num_parts, workspace=dec.workspace)
         if ev is not None:
             ev[1].record(stream)
-        api.combine(dec.workspace, d["seq_lens"], dec.max_pages, dims, dec.num_parts,
-                    o_lat=dec.o_lat, lse_out=dec.lse)
-        api.absorb_out(dec.o_lat, d["w_uv"], dims, out=dec.out)
+        if a.unfused:
+            api.combine(dec.workspace, d["seq_lens"], dec.max_pages, dims, dec.num_parts,
+                        o_lat=dec.o_lat, lse_out=dec.lse)
+            api.absorb_out(dec.o_lat, d["w_uv"], dims, out=dec.out)
+        else:
+            api.combine_absorb_out(dec.workspace, d["seq_lens"], dec.max_pages, dims,
+                                   dec.num_parts, d["w_uv"], out=dec.out, lse_out=dec.lse)
 
     def barrier():
         if world > 1:
@@ -348,12 +355,15 @@ def main():
                        "seq_len": w.seq_len or list(w.ragged), "heads": w.heads,
                        "kv_tokens_per_step": tokens_per_step, "num_parts": dec.num_parts,
                        "l2": "inputs larger than L2 (latent cache %.2f GB), no flush" % (kv_bytes / 1e9),
-                       "parallelism": "replicas" if world > 1 else "single"},
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "step_calls": ["mla_absorb_q", "mla_decode_splitkv"] +
+                                     (["mla_combine", "mla_absorb_out"] if a.unfused
+                                      else ["mla_combine_absorb_out"])},
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks,
-            "gpu_launches": 4 * a.steps}
+            "gpu_launches": (4 if a.unfused else 3) * a.steps}
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, a.cpu_seconds)
     if rank == 0:

@@ -159,6 +159,26 @@ mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t works
 mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w_uv, void *out,
                           int32_t num_tokens, void *stream);
 
+/*
+ * Combine and absorb-out in one call (the merge of mla_combine followed by the
+ * W_UV product of mla_absorb_out, "MHA2MLA" §2.1), without writing o_lat:
+ *   L = logsumexp_s lse_s,  o_lat = sum_s exp(lse_s - L) o_s   (as mla_combine)
+ *   out[t, h, :] = bf16( sum_c bf16(o_lat[t, h, c]) * w_uv[h, c, :] )
+ * over the tokens t = b * n_q + i of the batch. Arguments as mla_combine, plus
+ * w_uv [H, d_latent, d_v] bf16 and out [batch * n_q, H, d_v] bf16 (device,
+ * caller-owned, 16-byte aligned); lse_out [batch * n_q, H] fp32 may be NULL.
+ * The K sum may split d_latent into 128-channel parts reduced in a fixed
+ * order, so the result can differ from mla_combine + mla_absorb_out in the
+ * last bit of a bf16 output; repeated calls are bitwise identical.
+ * Supported: d_v <= 128, d_latent 64, 128 or a multiple of 128 up to 1024
+ * (MLA_ERR_UNSUPPORTED otherwise); MLA_ERR_INVALID_ARG on null/misaligned
+ * pointers or a workspace smaller than mla_decode_workspace_bytes.
+ */
+mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
+                                  size_t workspace_bytes, const int32_t *seq_lens,
+                                  int32_t max_pages_per_seq, int32_t batch, int32_t num_parts,
+                                  const void *w_uv, void *out, float *lse_out, void *stream);
+
 /* Synchronises `stream`, returns in *code (host pointer) the first error a
  * kernel of this library recorded on the current device since the last call
  * (MLA_OK if none), and clears it. */

@@ -154,6 +154,20 @@ def get_device_error(stream=None):
     return code.value
 
 
+def combine_absorb_out(workspace, seq_lens, max_pages, dims, num_parts, w_uv, out=None,
+                       lse_out=None, stream=None):
+    """Combine and absorb-out in one call: out [B, n_q, H, d_v] bf16."""
+    B = seq_lens.shape[0]
+    if out is None:
+        out = torch.empty((B, dims.n_q, dims.num_heads, dims.d_v), dtype=torch.bfloat16,
+                          device=workspace.device)
+    _b.check(_b.lib.mla_combine_absorb_out(ctypes.byref(dims), _ptr(workspace), workspace.numel(),
+                                           _ptr(seq_lens), max_pages, B, num_parts, _ptr(w_uv),
+                                           _ptr(out), _ptr(lse_out), _stream(stream)),
+             "mla_combine_absorb_out")
+    return out
+
+
 def debug_gather(pool, block_table, seq_lens, max_len, out=None, stream=None):
     """Gathered rows of a [pages, 64, width] (possibly channel-sliced) pool:
     out[b, t, :] = pool[block_table[b, t // 64], t % 64, :] for t < seq_lens[b]

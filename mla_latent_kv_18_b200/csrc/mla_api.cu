@@ -84,7 +84,9 @@ mla_status device_ready() {
             cudaFuncSetAttribute(mla::proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::proj_smem_bytes(256)) != cudaSuccess ||
             cudaFuncSetAttribute(mla::gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 64 * kGatherMaxWidth * 2) != cudaSuccess) {
+                                 64 * kGatherMaxWidth * 2) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::co_smem_bytes(128, mla::kCoMaxNT)) != cudaSuccess) {
             st.status = MLA_ERR_CUDA;
             return;
         }
@@ -447,6 +449,71 @@ mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const 
     if (st != MLA_OK) return st;
     return mla_combine(dims, scratch, MLA_NOALLOC_SCRATCH_BYTES, seq_lens, max_pages_per_seq, batch,
                        num_parts, o_lat, lse_out, stream);
+}
+
+mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
+                                  size_t workspace_bytes, const int32_t *seq_lens,
+                                  int32_t max_pages_per_seq, int32_t batch, int32_t num_parts,
+                                  const void *w_uv, void *out, float *lse_out, void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0) return MLA_ERR_INVALID_ARG;
+    const int32_t dc = dims->d_latent;
+    if (dims->d_v > 128 || !(dc == 64 || dc == 128 || (dc % 128 == 0 && dc <= 1024)))
+        return MLA_ERR_UNSUPPORTED;
+    if (batch == 0) return MLA_OK;
+    if (!workspace || !seq_lens || !w_uv || !out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(w_uv, 16) || !aligned(out, 16) || !aligned(seq_lens, 4) ||
+        (lse_out && !aligned(lse_out, 4)))
+        return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_decode_workspace_bytes(dims, batch, num_parts)) return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    const int64_t R = static_cast<int64_t>(dims->n_q) * dims->num_heads;
+    const int64_t slots = static_cast<int64_t>(batch) + num_parts;
+    const int64_t T64 = static_cast<int64_t>(batch) * dims->n_q;
+    if (T64 > (int64_t(1) << 30)) return MLA_ERR_UNSUPPORTED;
+    const int32_t T = static_cast<int32_t>(T64);
+    const int32_t NT = 16;   // tokens per CTA: the smallest MMA N, for the most CTAs (W_UV re-reads hit L2)
+    const int32_t KS = dc >= 256 ? dc / 128 : 1;
+    const int32_t KC = dc / KS;
+    CUtensorMap mw;
+    if ((st = map_3d(&mw, w_uv, dims->d_v, dc, dims->num_heads, uint64_t(dims->d_v) * 2,
+                     uint64_t(dc) * dims->d_v * 2, 64, 64, 1)) != MLA_OK)
+        return st;
+    mla::CombineOutArgs a;
+    a.o_part = static_cast<const float *>(workspace);
+    a.lse_part = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) +
+                                                 round_up(slots * R * dc * 4, 256));
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse_out = lse_out;
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.batch = batch;
+    a.max_pages = max_pages_per_seq;
+    a.n_q = dims->n_q;
+    a.H = dims->num_heads;
+    a.rows = static_cast<int32_t>(R);
+    a.d_c = dc;
+    a.d_v = dims->d_v;
+    a.tile_tokens = tile_tokens(variant_of(dims));
+    a.num_parts = num_parts;
+    a.T = T;
+    a.NT = NT;
+    a.KS = KS;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(dims->num_heads * KS), static_cast<unsigned>((T + NT - 1) / NT));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = mla::co_smem_bytes(KC, NT);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(KS);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla::combine_out_kernel, mw, a) != cudaSuccess) return MLA_ERR_CUDA;
+    return launch_status();
 }
 
 mla_status mla_debug_gather(const mla_pool *pool, int32_t width, int32_t num_pages,

@@ -278,6 +278,221 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
 // One block waits on a barrier nothing completes; the bounded wait runs out
 // after timeout_ns and records kErrTimeout.
 // ---------------------------------------------------------------------------
+// Fused combine + absorb-out: the split-KV merge followed by the per-head W_UV
+// product ("MHA2MLA" page §2.1, v = c_kv W_uv applied once to the latent
+// result):
+//   o_lat[t, h, :] = sum_s exp(lse_s - L) o_s[t, h, :],  L = logsumexp_s lse_s
+//   out[t, h, :]   = bf16(o_lat[t, h, :]) W_UV[h]        (fp32 accumulation)
+// The merged row never goes back to HBM: it is rounded to bf16 straight into
+// the MMA's shared-memory operand.
+// grid (H * KS, ceil(T / NT)), clusters of KS CTAs along x, 128 threads. CTA q
+// of head h's cluster takes latent channels [q * KC, (q + 1) * KC), KC = d_c / KS
+// (64 or 128): it merges those channels of every token of its tile (same
+// arithmetic and slot order as combine_kernel), streams the matching KC rows of
+// W_UV[h] by TMA (MN-major, overlapped with the merge) and computes the partial
+// D[col, t] = W^T[col, k] x^T[k, t] in tensor memory. The KS partial tiles are
+// added in rank order over distributed shared memory, each CTA finishing
+// 128 / KS output columns.
+// ---------------------------------------------------------------------------
+struct CombineOutArgs {
+    const float *o_part;     // [slots, R, d_c]
+    const float *lse_part;   // [slots, R]
+    const int32_t *seq_lens;
+    __nv_bfloat16 *out;      // [T, H, d_v]
+    float *lse_out;          // [T, H] or null
+    int64_t timeout_ns;
+    int32_t batch, max_pages, n_q, H, rows, d_c, d_v, tile_tokens, num_parts, T, NT, KS;
+};
+
+constexpr int kCoMaxNT = 64;
+__host__ __device__ constexpr uint32_t co_smem_bytes(int KC, int NT) {
+    return static_cast<uint32_t>(KC / 64) * 16384u            // W_UV rows: two 64-column atoms per K block
+           + static_cast<uint32_t>(KC / 64) * NT * 128u        // merged rows (bf16, K-major, swizzled)
+           + static_cast<uint32_t>(NT) * 128u * 4u             // partial D tile [t][col] fp32
+           + 1024u /* barriers */ + 1024u /* alignment */;
+}
+
+__global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant__ CUtensorMap map_w,
+                                                          const CombineOutArgs a) {
+    extern __shared__ uint8_t co_smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(co_smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KS = a.KS, NT = a.NT;
+    const uint32_t q = (KS > 1) ? ptx::cluster_ctarank() : 0u;
+    const int h = blockIdx.x / KS;
+    const int t0 = blockIdx.y * NT;
+    const int KC = a.d_c / KS;
+    const int KB = KC / 64;
+    const int nt = min(NT, a.T - t0);
+    const uint32_t w_s = base;
+    const uint32_t x_s = w_s + KB * 16384u;
+    const uint32_t part_s = x_s + KB * NT * 128u;
+    const uint32_t bar_s = part_s + NT * 128u * 4u;
+    uint8_t *bar_p = co_smem_raw + (bar_s - raw_base);
+    const uint32_t wfull = bar_s, done = bar_s + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_p + 16);
+    int32_t *abort_flag = reinterpret_cast<int32_t *>(bar_p + 20);
+    uint32_t tcols = 32;
+    while (tcols < static_cast<uint32_t>(NT)) tcols <<= 1;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(wfull, 1);
+        ptx::mbar_init(done, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        // W_UV[h] rows [q * KC, (q + 1) * KC): issued first, lands during the merge
+        ptx::mbar_arrive_expect_tx(wfull, KB * 16384u);
+        for (int kb = 0; kb < KB; ++kb) {
+            const int k0 = static_cast<int>(q) * KC + kb * 64;
+            ptx::tma_load_3d(w_s + kb * 16384u, &map_w, wfull, 0, k0, h);
+            ptx::tma_load_3d(w_s + kb * 16384u + 8192u, &map_w, wfull, 64, k0, h);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
+        ptx::tmem_relinquish<1>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int32_t *abort_v = abort_flag;
+
+    // ---- merge: warp w takes tokens w, w + 4, ...; lane covers 4 channels
+    const int c_loc = 4 * lane;   // channel within this CTA's KC
+    for (int tt = warp; tt < NT; tt += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (tt < nt) {
+            const int t = t0 + tt;
+            const int32_t b = t / a.n_q;
+            const int r = (t - b * a.n_q) * a.H + h;
+            int64_t sbase = 0, cnt = 0;
+            sequence_slots(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts, b,
+                           &sbase, &cnt);
+            const float *lse_r = a.lse_part + sbase * a.rows + r;
+            float m = -INFINITY;
+            for (int64_t s = lane; s < cnt; s += 32) m = fmaxf(m, lse_r[s * a.rows]);
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float z = 0.f;
+            if (m > -INFINITY)
+                for (int64_t s = lane; s < cnt; s += 32) z += __expf(lse_r[s * a.rows] - m);
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            const float L = (m > -INFINITY) ? m + __logf(z) : -INFINITY;
+            if (a.lse_out && q == 0 && lane == 0) a.lse_out[static_cast<int64_t>(t) * a.H + h] = L;
+            if (m > -INFINITY && c_loc < KC) {
+                const float *o_r = a.o_part + (sbase * a.rows + r) * a.d_c + q * KC + c_loc;
+                const int64_t slot_stride = static_cast<int64_t>(a.rows) * a.d_c;
+                constexpr int U = 8;
+                for (int64_t s0 = 0; s0 < cnt; s0 += U) {
+                    float w[U];
+                    float4 v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int64_t s = s0 + u;
+                        w[u] = 0.f;
+                        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (s < cnt) {
+                            const float ls = lse_r[s * a.rows];
+                            w[u] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
+                            v[u] = *reinterpret_cast<const float4 *>(o_r + s * slot_stride);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        acc.x = fmaf(w[u], v[u].x, acc.x);
+                        acc.y = fmaf(w[u], v[u].y, acc.y);
+                        acc.z = fmaf(w[u], v[u].z, acc.z);
+                        acc.w = fmaf(w[u], v[u].w, acc.w);
+                    }
+                }
+            }
+        }
+        if (c_loc < KC) {   // bf16 into the K-major, 128-byte-swizzled operand tile
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            const int kb = c_loc >> 6, within = c_loc & 63;
+            const uint32_t addr = x_s + kb * NT * 128u + sw128(tt, within >> 3) + ((within & 7) >> 2) * 8u;
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr),
+                         "r"(*reinterpret_cast<uint32_t *>(&lo)), "r"(*reinterpret_cast<uint32_t *>(&hi))
+                         : "memory");
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+
+    // ---- tensor cores: D[col, t] = sum_k W[k, col] x[t, k] over this CTA's KC rows
+    if (warp == 1 && ptx::elect_one()) {
+        if (wait_bounded<false>(wfull, 0, abort_v, a.timeout_ns)) {
+            ptx::tc_fence_after();
+            const uint32_t idesc = ptx::idesc_bf16(128, NT, 1, 0);
+            for (int kb = 0; kb < KB; ++kb) {
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = ptx::smem_desc(w_s + kb * 16384u + kk * 2048u, 64 * 128, 1024,
+                                                       ptx::kSwizzle128B);
+                    const uint64_t bd = ptx::smem_desc(x_s + kb * NT * 128u + kk * 32u, 16, 1024,
+                                                       ptx::kSwizzle128B);
+                    ptx::mma_bf16_ss<1>(tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+                }
+            }
+        }
+        ptx::mma_commit(done);
+    }
+    const bool ok = wait_bounded<false>(done, 0, abort_v, a.timeout_ns) && !*abort_v;
+    ptx::tc_fence_after();
+    const int col = 32 * warp + lane;   // TMEM lane = output column
+    if (KS == 1) {
+        if (ok) {
+            for (int c0 = 0; c0 < NT; c0 += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, v);
+                ptx::tmem_wait_ld();
+                if (col < a.d_v) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = c0 + j;
+                        if (t < nt)
+                            a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.d_v + col] =
+                                __float2bfloat16_rn(__uint_as_float(v[j]));
+                    }
+                }
+            }
+        }
+    } else {
+        // partial tile to shared memory as [t][col], then the rank-ordered sum
+        for (int c0 = 0; c0 < NT; c0 += 32) {
+            uint32_t v[32];
+            ptx::tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = c0 + j;
+                if (t < NT) {
+                    const float val = ok ? __uint_as_float(v[j]) : 0.f;
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(part_s + (t * 128u + col) * 4u), "f"(val)
+                                 : "memory");
+                }
+            }
+        }
+        ptx::cluster_sync();
+        const int cw = 128 / KS;   // output columns finished by this CTA
+        for (int idx = threadIdx.x; idx < nt * cw; idx += 128) {
+            const int t = idx / cw, cl = static_cast<int>(q) * cw + (idx - t * cw);
+            const uint32_t off = part_s + (t * 128u + cl) * 4u;
+            float sum = 0.f;
+            for (int rk = 0; rk < KS; ++rk) sum += ptx::ld_shared_cluster_f32(ptx::mapa(off, rk));
+            if (cl < a.d_v)
+                a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.d_v + cl] = __float2bfloat16_rn(sum);
+        }
+        ptx::cluster_sync();   // peers read this CTA's tile until here
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc<1>(tmem, tcols);
+}
+
+// ---------------------------------------------------------------------------
 // Debug gather: the page lookup of the decode kernels (token t of sequence b
 // is row t % 64 of page block_table[b][t / 64], "MLA operator design" page §3)
 // through a TMA pool descriptor like theirs, written out densely.

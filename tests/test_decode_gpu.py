@@ -276,6 +276,39 @@ def test_gather_bad_page_id_sets_device_error(api):
     assert api.get_device_error() == 0
 
 
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("dsv3", dict(batch=4, seq_len=3000)),
+                                     ("dsv3", dict(batch=80, heads=16, seq_len=200)),
+                                     ("ragged", dict(batch=6, heads=128, ragged=(64, 4000))),
+                                     ("retrofit", dict(batch=9, seq_len=700))])
+def test_fused_combine_absorb_out(api, name, kw):
+    """mla_combine_absorb_out against the oracle's absorb-out of the GPU's own
+    merged rows (the same definition, composed) and end to end against the fp64
+    absorbed path; its lse equals mla_combine's bit for bit, its output stays
+    within one bf16 rounding of mla_combine + mla_absorb_out, and a repeat call
+    is bitwise identical."""
+    w = workload(name, **kw)
+    inp = make_inputs(w, seed=15)
+    d = to_device(inp, "cuda")
+    r = _run(api, d)
+    dims, ws, P = r["dims"], r["ws"], r["num_parts"]
+    lse = torch.empty_like(r["lse"])
+    out = api.combine_absorb_out(ws, d["seq_lens"], d["block_table"].shape[1], dims, P, d["w_uv"],
+                                 lse_out=lse)
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    assert torch.equal(lse, r["lse"])
+    out_ref = oracle.absorb_out(r["o_lat"].cpu(), inp["w_uv"])   # fp64 over the same bf16 o_lat
+    _check(_f64(out), out_ref, "fused out vs oracle absorb-out")
+    _check_rounded(_f64(out), _f64(r["out"]), "fused vs unfused")
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    sel = _sample_rows(w, 256, 15)
+    ab, _, _ = oracle.decode_absorbed(*args, sel=sel)
+    _check(_f64(out).reshape(-1, w.d_v)[sel], ab.reshape(-1, w.d_v)[sel], "fused out vs absorbed")
+    again = api.combine_absorb_out(ws, d["seq_lens"], d["block_table"].shape[1], dims, P, d["w_uv"])
+    assert torch.equal(again, out)
+
+
 def test_repeat_calls_are_bitwise_identical(api):
     w = workload("ragged", batch=8, heads=128, ragged=(500, 5000))
     inp_d = to_device(make_inputs(w, seed=9), "cuda")
