@@ -170,8 +170,8 @@ mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w
  * The K sum may split d_latent into 128-channel parts reduced in a fixed
  * order, so the result can differ from mla_combine + mla_absorb_out in the
  * last bit of a bf16 output; repeated calls are bitwise identical.
- * Supported: d_v <= 128, d_latent 64, 128 or a multiple of 128 up to 1024
- * (MLA_ERR_UNSUPPORTED otherwise); MLA_ERR_INVALID_ARG on null/misaligned
+ * Supported: d_v <= 128, d_latent 64, 128 or a multiple of 128 up to 1024,
+ * num_parts < 160 (MLA_ERR_UNSUPPORTED otherwise); MLA_ERR_INVALID_ARG on null/misaligned
  * pointers or a workspace smaller than mla_decode_workspace_bytes.
  */
 mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,

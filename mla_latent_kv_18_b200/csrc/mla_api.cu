@@ -458,6 +458,7 @@ mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
     mla_status st = check_dims(dims, true);
     if (st != MLA_OK) return st;
     if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0) return MLA_ERR_INVALID_ARG;
+    if (num_parts >= mla::kCoMaxSlots) return MLA_ERR_UNSUPPORTED;   // slots per sequence <= num_parts + 1
     const int32_t dc = dims->d_latent;
     if (dims->d_v > 128 || !(dc == 64 || dc == 128 || (dc % 128 == 0 && dc <= 1024)))
         return MLA_ERR_UNSUPPORTED;

@@ -59,6 +59,55 @@ __device__ inline void sequence_slots(const int32_t *seq_lens, int32_t batch, in
     }
 }
 
+// (slot_base, slot_count) of every sequence b in [b_lo, b_hi] into
+// base[b - b_lo], cnt[b - b_lo] (shared memory); warp-wide, one pass.
+__device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t batch, int32_t max_pages,
+                                            int32_t n_q, int32_t tile_tokens, int64_t P, int32_t b_lo,
+                                            int32_t b_hi, int64_t *base, int32_t *cnt) {
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    int64_t N = 0;
+    for (int32_t b0 = 0; b0 < batch; b0 += 32) {
+        const int32_t bb = b0 + lane;
+        int64_t n = 0;
+        if (bb < batch) n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        N += n;
+    }
+    for (int32_t b = b_lo + lane; b <= b_hi; b += 32) {
+        base[b - b_lo] = 0;
+        cnt[b - b_lo] = 0;
+    }
+    if (N == 0) return;
+    P = parts_in_use(P, N);
+    int64_t O = 0, S = 0;
+    for (int32_t b0 = 0; b0 <= b_hi; b0 += 32) {
+        const int32_t bb = b0 + lane;
+        int64_t n = 0;
+        if (bb < batch && bb <= b_hi)
+            n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        int64_t incl = n;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int64_t Ob = O + incl - n;
+        int64_t ns = 0;
+        if (n > 0) ns = part_of_tile(Ob + n - 1, N, P) - part_of_tile(Ob, N, P) + 1;
+        int64_t sincl = ns;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t v = __shfl_up_sync(0xffffffffu, sincl, o);
+            if (lane >= o) sincl += v;
+        }
+        if (bb >= b_lo && bb <= b_hi) {
+            base[bb - b_lo] = S + sincl - ns;
+            cnt[bb - b_lo] = static_cast<int32_t>(ns);
+        }
+        O += __shfl_sync(0xffffffffu, incl, 31);
+        S += __shfl_sync(0xffffffffu, sincl, 31);
+    }
+}
+
 struct CombineArgs {
     const float *o_part;     // [slots, R, d_c]
     const float *lse_part;   // [slots, R]
@@ -305,11 +354,15 @@ struct CombineOutArgs {
 };
 
 constexpr int kCoMaxNT = 64;
+constexpr int kCoMaxSlots = 160;   // partial slots per sequence (num_parts + 1 at most)
 __host__ __device__ constexpr uint32_t co_smem_bytes(int KC, int NT) {
     return static_cast<uint32_t>(KC / 64) * 16384u            // W_UV rows: two 64-column atoms per K block
            + static_cast<uint32_t>(KC / 64) * NT * 128u        // merged rows (bf16, K-major, swizzled)
            + static_cast<uint32_t>(NT) * 128u * 4u             // partial D tile [t][col] fp32
-           + 1024u /* barriers */ + 1024u /* alignment */;
+           + static_cast<uint32_t>(NT) * kCoMaxSlots * 4u      // merge weights [t][slot]
+           + static_cast<uint32_t>(NT) * 16u                   // per token: first slot, count, row
+           + static_cast<uint32_t>(NT) * 16u                   // per sequence: first slot, count
+           + 128u /* barriers */ + 1024u /* alignment */;
 }
 
 __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant__ CUtensorMap map_w,
@@ -328,7 +381,16 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     const uint32_t w_s = base;
     const uint32_t x_s = w_s + KB * 16384u;
     const uint32_t part_s = x_s + KB * NT * 128u;
-    const uint32_t bar_s = part_s + NT * 128u * 4u;
+    const uint32_t wts_s = part_s + NT * 128u * 4u;
+    const uint32_t tok_s = wts_s + NT * kCoMaxSlots * 4u;
+    const uint32_t seq_s = tok_s + NT * 16u;
+    const uint32_t bar_s = seq_s + NT * 16u;
+    int64_t *seq_base = reinterpret_cast<int64_t *>(co_smem_raw + (seq_s - raw_base));
+    int32_t *seq_cnt = reinterpret_cast<int32_t *>(co_smem_raw + (seq_s - raw_base) + NT * 8);
+    float *wts = reinterpret_cast<float *>(co_smem_raw + (wts_s - raw_base));
+    int64_t *tok_base = reinterpret_cast<int64_t *>(co_smem_raw + (tok_s - raw_base));
+    int32_t *tok_cnt = reinterpret_cast<int32_t *>(co_smem_raw + (tok_s - raw_base) + NT * 8);
+    int32_t *tok_row = reinterpret_cast<int32_t *>(co_smem_raw + (tok_s - raw_base) + NT * 12);
     uint8_t *bar_p = co_smem_raw + (bar_s - raw_base);
     const uint32_t wfull = bar_s, done = bar_s + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_p + 16);
@@ -359,63 +421,136 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     volatile int32_t *abort_v = abort_flag;
 
-    // ---- merge: warp w takes tokens w, w + 4, ...; lane covers 4 channels
-    const int c_loc = 4 * lane;   // channel within this CTA's KC
-    for (int tt = warp; tt < NT; tt += 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (tt < nt) {
+    // ---- merge, phase 1: the slots of the tile's sequences (one warp, one
+    // pass), then eight threads per token find L and the weights exp(lse_s - L)
+    // with the same arithmetic and the same addition tree as combine_kernel
+    const int32_t b_lo = t0 / a.n_q, b_hi = (t0 + nt - 1) / a.n_q;   // at most NT sequences
+    if (warp == 0)
+        sequence_slots_range(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts,
+                             b_lo, b_hi, seq_base, seq_cnt);
+    __syncthreads();
+    for (int tt = threadIdx.x >> 3; tt < NT; tt += 16) {
+        const int sub = threadIdx.x & 7;
+        const bool live = tt < nt;
+        int64_t sbase = 0;
+        int cnt = 0, r = 0;
+        if (live) {
             const int t = t0 + tt;
             const int32_t b = t / a.n_q;
-            const int r = (t - b * a.n_q) * a.H + h;
-            int64_t sbase = 0, cnt = 0;
-            sequence_slots(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts, b,
-                           &sbase, &cnt);
-            const float *lse_r = a.lse_part + sbase * a.rows + r;
-            float m = -INFINITY;
-            for (int64_t s = lane; s < cnt; s += 32) m = fmaxf(m, lse_r[s * a.rows]);
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float z = 0.f;
-            if (m > -INFINITY)
-                for (int64_t s = lane; s < cnt; s += 32) z += __expf(lse_r[s * a.rows] - m);
-            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            const float L = (m > -INFINITY) ? m + __logf(z) : -INFINITY;
-            if (a.lse_out && q == 0 && lane == 0) a.lse_out[static_cast<int64_t>(t) * a.H + h] = L;
-            if (m > -INFINITY && c_loc < KC) {
-                const float *o_r = a.o_part + (sbase * a.rows + r) * a.d_c + q * KC + c_loc;
-                const int64_t slot_stride = static_cast<int64_t>(a.rows) * a.d_c;
-                constexpr int U = 8;
-                for (int64_t s0 = 0; s0 < cnt; s0 += U) {
-                    float w[U];
-                    float4 v[U];
+            r = (t - b * a.n_q) * a.H + h;
+            sbase = seq_base[b - b_lo];
+            cnt = seq_cnt[b - b_lo];
+        }
+        const float *lse_r = a.lse_part + sbase * a.rows + r;
+        // thread sub stands for lanes sub, sub + 8, sub + 16, sub + 24 of a warp
+        // that strides the slots by 32; the first 32 slots' values stay in
+        // registers (one load round), later ones are read again
+        float lv[4];
 #pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int64_t s = s0 + u;
-                        w[u] = 0.f;
-                        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (s < cnt) {
-                            const float ls = lse_r[s * a.rows];
-                            w[u] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
-                            v[u] = *reinterpret_cast<const float4 *>(o_r + s * slot_stride);
-                        }
-                    }
+        for (int j = 0; j < 4; ++j) {
+            const int s = sub + 8 * j;
+            lv[j] = (s < cnt) ? lse_r[static_cast<int64_t>(s) * a.rows] : -INFINITY;
+        }
+        float mv[4] = {lv[0], lv[1], lv[2], lv[3]};
 #pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        acc.x = fmaf(w[u], v[u].x, acc.x);
-                        acc.y = fmaf(w[u], v[u].y, acc.y);
-                        acc.z = fmaf(w[u], v[u].z, acc.z);
-                        acc.w = fmaf(w[u], v[u].w, acc.w);
-                    }
-                }
+        for (int j = 0; j < 4; ++j)
+            for (int s = sub + 8 * j + 32; s < cnt; s += 32)
+                mv[j] = fmaxf(mv[j], lse_r[static_cast<int64_t>(s) * a.rows]);
+        float m = fmaxf(fmaxf(mv[0], mv[2]), fmaxf(mv[1], mv[3]));
+        for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float zv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (m > -INFINITY) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (sub + 8 * j < cnt) zv[j] = __expf(lv[j] - m);
+                for (int s = sub + 8 * j + 32; s < cnt; s += 32)
+                    zv[j] += __expf(lse_r[static_cast<int64_t>(s) * a.rows] - m);
             }
         }
-        if (c_loc < KC) {   // bf16 into the K-major, 128-byte-swizzled operand tile
-            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-            const int kb = c_loc >> 6, within = c_loc & 63;
-            const uint32_t addr = x_s + kb * NT * 128u + sw128(tt, within >> 3) + ((within & 7) >> 2) * 8u;
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr),
-                         "r"(*reinterpret_cast<uint32_t *>(&lo)), "r"(*reinterpret_cast<uint32_t *>(&hi))
-                         : "memory");
+        // the 32-lane xor tree: +16, +8 locally, then +4, +2, +1 across the 8 threads
+        float z = (zv[0] + zv[2]) + (zv[1] + zv[3]);
+        for (int o = 4; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        const float L = (m > -INFINITY) ? m + __logf(z) : -INFINITY;
+        if (live && a.lse_out && q == 0 && sub == 0)
+            a.lse_out[static_cast<int64_t>(t0 + tt) * a.H + h] = L;
+        if (m == -INFINITY || cnt > kCoMaxSlots) cnt = 0;   // nothing to merge (host caps the slots)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int s = sub + 8 * j;
+            if (s < cnt) wts[tt * kCoMaxSlots + s] = (lv[j] > -INFINITY) ? __expf(lv[j] - L) : 0.f;
+        }
+        for (int s = sub + 32; s < cnt; s += 8) {
+            const float ls = lse_r[static_cast<int64_t>(s) * a.rows];
+            wts[tt * kCoMaxSlots + s] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
+        }
+        if (sub == 0) {
+            tok_base[tt] = sbase;
+            tok_cnt[tt] = cnt;
+            tok_row[tt] = r;
+        }
+    }
+    __syncthreads();
+    // ---- merge, phase 2: items (token, 4 channels), all loads of a slot step
+    // issued together; slots are added in order, as in combine_kernel
+    {
+        const int chunks = KC / 4;
+        constexpr int IT = 4;   // items per thread (NT * chunks <= 16 * 32 = 512 = 4 x 128)
+        const int64_t slot_stride = static_cast<int64_t>(a.rows) * a.d_c;
+        for (int i0 = threadIdx.x; i0 < NT * chunks; i0 += IT * 128) {
+            float4 acc[IT];
+            const float *src[IT];
+            int cnt_i[IT], tt_i[IT];
+            int maxc = 0;
+#pragma unroll
+            for (int u = 0; u < IT; ++u) {
+                acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                const int i = i0 + u * 128;
+                tt_i[u] = i / chunks;
+                const bool live = i < NT * chunks;
+                cnt_i[u] = live ? tok_cnt[tt_i[u]] : 0;
+                src[u] = live ? a.o_part + (tok_base[tt_i[u]] * a.rows + tok_row[tt_i[u]]) * a.d_c +
+                                    q * KC + 4 * (i - tt_i[u] * chunks)
+                              : a.o_part;
+                maxc = max(maxc, cnt_i[u]);
+            }
+            constexpr int SS = 4;   // slots per step
+            for (int s = 0; s < maxc; s += SS) {
+                float4 v[IT][SS];
+                float w[IT][SS];
+#pragma unroll
+                for (int u = 0; u < IT; ++u)
+#pragma unroll
+                    for (int e = 0; e < SS; ++e) {
+                        const bool on = s + e < cnt_i[u];
+                        v[u][e] = on ? *reinterpret_cast<const float4 *>(src[u] + (s + e) * slot_stride)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                        w[u][e] = on ? wts[tt_i[u] * kCoMaxSlots + s + e] : 0.f;
+                    }
+#pragma unroll
+                for (int u = 0; u < IT; ++u)
+#pragma unroll
+                    for (int e = 0; e < SS; ++e) {
+                        if (s + e < cnt_i[u]) {
+                            acc[u].x = fmaf(w[u][e], v[u][e].x, acc[u].x);
+                            acc[u].y = fmaf(w[u][e], v[u][e].y, acc[u].y);
+                            acc[u].z = fmaf(w[u][e], v[u][e].z, acc[u].z);
+                            acc[u].w = fmaf(w[u][e], v[u][e].w, acc[u].w);
+                        }
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < IT; ++u) {   // bf16 into the K-major, 128-byte-swizzled operand tile
+                const int i = i0 + u * 128;
+                if (i >= NT * chunks) continue;
+                const int c_loc = 4 * (i - tt_i[u] * chunks);
+                __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+                const int kb = c_loc >> 6, within = c_loc & 63;
+                const uint32_t addr = x_s + kb * NT * 128u + sw128(tt_i[u], within >> 3) + ((within & 7) >> 2) * 8u;
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr),
+                             "r"(*reinterpret_cast<uint32_t *>(&lo)), "r"(*reinterpret_cast<uint32_t *>(&hi))
+                             : "memory");
+            }
         }
     }
     ptx::fence_proxy_async_smem();
