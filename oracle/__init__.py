@@ -46,6 +46,8 @@ def _load():
                                              P, i32, P, i32, i32, P, i64, P, P]
         lib.oracle_combine.argtypes = [i64, i32, i32, P, P, P, P]
         lib.oracle_absorb_out.argtypes = [i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_rope.argtypes = [i32, i32, i32, P, P, ctypes.c_double, P]
+        lib.oracle_rope.restype = i32
         for name in ("oracle_gather", "oracle_decode_decompress", "oracle_absorb_q",
                      "oracle_attend_latent", "oracle_combine", "oracle_absorb_out"):
             getattr(lib, name).restype = i32
@@ -168,6 +170,20 @@ def absorb_q(q_c, w_uk):
     T = int(np.prod(lead)) if lead else 1
     out = np.zeros(lead + (H, d_c), dtype=np.float64)
     _check(_load().oracle_absorb_q(T, H, d_n, d_c, _p(qc), _p(wuk), _p(out)), "absorb_q")
+    return out
+
+
+def rope(q_r, positions, theta=10000.0):
+    """Rotary embedding of the RoPE part, fp64: consecutive pairs (2i, 2i+1)
+    turn by positions[t] * theta^(-2i/d_r). q_r [..., H, d_r] bf16, positions
+    [...] int (one per token) -> [..., H, d_r]."""
+    x = _bits(q_r)
+    lead, (H, d_r) = x.shape[:-2], x.shape[-2:]
+    T = int(np.prod(lead)) if lead else 1
+    pos = _i32(np.asarray(positions).reshape(-1))
+    assert pos.size == T
+    out = np.zeros(lead + (H, d_r), dtype=np.float64)
+    _check(_load().oracle_rope(T, H, d_r, _p(x), _p(pos), float(theta), _p(out)), "rope")
     return out
 
 

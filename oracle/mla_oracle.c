@@ -199,6 +199,38 @@ int oracle_absorb_q(int T, int H, int d_n, int d_c, const uint16_t *q_c, const u
 }
 
 /*
+ * Rotary position embedding of the query's RoPE part ("MHA2MLA" page §3.2,
+ * rope_theta 10000; the "MLA operator design" page §3 computes it in fp32,
+ * this reference in fp64). Consecutive pairs (2i, 2i + 1) of x[t][h][:] turn
+ * by the angle a = pos[t] * theta^(-2i / d_r):
+ *   y[2i]     = x[2i] cos(a) - x[2i + 1] sin(a)
+ *   y[2i + 1] = x[2i] sin(a) + x[2i + 1] cos(a)
+ * x [T,H,d_r] bf16, pos [T] int32 (>= 0), y [T,H,d_r] fp64. Returns -1 on a
+ * negative position or an odd d_r.
+ */
+int oracle_rope(int T, int H, int d_r, const uint16_t *x, const int32_t *pos, double theta,
+                double *y) {
+    if (d_r % 2 != 0 || theta <= 0.0) return -1;
+    for (int t = 0; t < T; ++t)
+        if (pos[t] < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t th = 0; th < (int64_t)T * H; ++th) {
+        const int t = (int)(th / H);
+        const uint16_t *xi = x + th * d_r;
+        double *yo = y + th * d_r;
+        for (int i = 0; i < d_r / 2; ++i) {
+            const double freq = pow(theta, -2.0 * i / d_r);
+            const double a = (double)pos[t] * freq;
+            const double c = cos(a), sn = sin(a);
+            const double x0 = bf16_to_f64(xi[2 * i]), x1 = bf16_to_f64(xi[2 * i + 1]);
+            yo[2 * i] = x0 * c - x1 * sn;
+            yo[2 * i + 1] = x0 * sn + x1 * c;
+        }
+    }
+    return 0;
+}
+
+/*
  * Attention in latent space (the absorbed score and value steps):
  *   s[t]   = scale * (sum_c Q[c] c_KV[t][c] + sum_j Q[d_c + j] k_R[t][j])
  *   o[c]   = sum_t softmax(s)[t] * c_KV[t][c]

@@ -448,3 +448,59 @@ def test_absorb_out_orientation_and_brute_force():
                                atol=1e-13)
     # fp64 input path agrees with the bf16 path on bf16-exact values
     np.testing.assert_array_equal(oracle.absorb_out(od, Wr), got)
+
+
+ROPE_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "rope_example.txt")
+
+
+def _kv(path):
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = (s.strip() for s in line.split("="))
+                vals[k] = float(v)
+    return vals
+
+
+def test_rope_worked_example():
+    """Hand-worked rotation (tests/golden/rope_example.txt): pins the pairing of
+    adjacent channels, the frequency exponent, the sign of the angle and the
+    position factor."""
+    v = _kv(ROPE_GOLDEN)
+    x = torch.tensor([[[1.0, 0.0, 0.0, 1.0]], [[1.0, 0.0, 0.0, 1.0]]], dtype=torch.bfloat16)
+    y = oracle.rope(x, [1, 3], theta=10000.0)
+    np.testing.assert_allclose(y[0, 0], [v["y0"], v["y1"], v["y2"], v["y3"]], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(y[1, 0], [v["z0"], v["z1"], v["z2"], v["z3"]], rtol=0, atol=1e-15)
+
+
+def test_rope_position_zero_is_identity_and_pair_norms_are_kept():
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(5, 3, 8, generator=g).to(torch.bfloat16)
+    pos = [0, 1, 7, 1000, 65535]
+    y = oracle.rope(x, pos)
+    xf = oracle.bf16_bits_to_f64(x).reshape(5, 3, 8)
+    assert np.array_equal(y[0], xf[0])
+    n_in = xf[..., 0::2] ** 2 + xf[..., 1::2] ** 2
+    n_out = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    np.testing.assert_allclose(n_out, n_in, rtol=1e-12, atol=0)
+
+
+@pytest.mark.parametrize("d_r", [8, 64])
+def test_rope_scores_depend_only_on_relative_position(d_r):
+    """<R_p x, R_q z> = <R_(p+s) x, R_(q+s) z>: the defining property of a
+    rotary embedding (rotations compose by adding angles)."""
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(1, 1, d_r, generator=g).to(torch.bfloat16).expand(4, 1, d_r).contiguous()
+    z = torch.randn(1, 1, d_r, generator=g).to(torch.bfloat16).expand(4, 1, d_r).contiguous()
+    p, q = 17, 5
+    for s in (1, 250, 40000):
+        rx = oracle.rope(x[:2], [p, p + s])
+        rz = oracle.rope(z[:2], [q, q + s])
+        d0 = float(np.dot(rx[0, 0], rz[0, 0]))
+        d1 = float(np.dot(rx[1, 0], rz[1, 0]))
+        assert abs(d0 - d1) <= 1e-9 * max(1.0, abs(d0))
+    # and it is not symmetric in p and q: the angle has a direction
+    ra, rb = oracle.rope(x[:2], [p, q]), oracle.rope(z[:2], [q, p])
+    assert abs(float(np.dot(ra[0, 0], rb[0, 0])) - float(np.dot(ra[1, 0], rb[1, 0]))) > 1e-6
