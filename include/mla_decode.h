@@ -152,6 +152,26 @@ mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t works
                        int32_t num_parts, void *o_lat, float *lse_out, void *stream);
 
 /*
+ * Absorb-in with the rotary embedding of the RoPE part fused in: as
+ * mla_absorb_q, except that q_r arrives unrotated and
+ *   q_out[t, h, d_latent + 2i]     = bf16(x0 cos(a) - x1 sin(a))
+ *   q_out[t, h, d_latent + 2i + 1] = bf16(x0 sin(a) + x1 cos(a))
+ * with (x0, x1) = q_r[t, h, 2i .. 2i + 1] and a = positions[t] *
+ * rope_theta^(-2i / d_rope) ("MHA2MLA" §3.2, rope_theta 10000; the "MLA
+ * operator design" page §3 computes RoPE in fp32: here the angle and its
+ * reduction are fp64, the rotation fp32). The pairing of adjacent channels is
+ * this library's reading of a convention the pages leave unstated.
+ * positions [num_tokens] int32 device (the token's absolute position, e.g.
+ * seq_len - n_q + i for query i of a sequence); a negative entry is treated as
+ * 0 and sets MLA_ERR_DEVICE_BOUNDS in the device error word. rope_theta must
+ * be finite and > 1 (MLA_ERR_INVALID_ARG otherwise). The latent part is
+ * identical to mla_absorb_q's.
+ */
+mla_status mla_absorb_q_rope(const mla_dims *dims, const void *q_c, const void *q_r,
+                             const void *w_uk, const int32_t *positions, float rope_theta,
+                             void *q_out, int32_t num_tokens, void *stream);
+
+/*
  * Absorb-out ("MHA2MLA" §2.1: v = c_kv W_uv, applied once to the latent result).
  *   out[t, h, :] = bf16( sum_c o_lat[t, h, c] * w_uv[h, c, :] )   (fp32 accumulation)
  * o_lat [T, H, d_latent] bf16, w_uv [H, d_latent, d_v] bf16, out [T, H, d_v] bf16.

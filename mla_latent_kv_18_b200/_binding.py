@@ -17,7 +17,8 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTS = ("mla_absorb_q", "mla_decode_num_parts", "mla_decode_workspace_bytes",
            "mla_decode_splitkv", "mla_combine", "mla_absorb_out", "mla_get_device_error",
            "mla_status_string", "mla_decode_plan", "mla_debug_wait_timeout",
-           "mla_decode_latent_noalloc", "mla_debug_gather", "mla_combine_absorb_out")
+           "mla_decode_latent_noalloc", "mla_debug_gather", "mla_combine_absorb_out",
+           "mla_absorb_q_rope")
 
 
 class MLADims(ctypes.Structure):
@@ -59,6 +60,7 @@ def _load():
         "mla_decode_latent_noalloc": (i32, [D, P, PL, PL, i32, P, i32, P, i32, i32, P, P, P]),
         "mla_debug_gather": (i32, [PL, i32, i32, P, i32, P, i32, i32, P, P]),
         "mla_combine_absorb_out": (i32, [D, P, sz, P, i32, i32, i32, P, P, P, P]),
+        "mla_absorb_q_rope": (i32, [D, P, P, P, P, ctypes.c_float, P, i32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -138,6 +138,19 @@ def combine(workspace, seq_lens, max_pages, dims, num_parts, o_lat=None, lse_out
     return o_lat, lse_out
 
 
+def absorb_q_rope(q_c, q_r, w_uk, dims, positions, theta=10000.0, out=None, stream=None):
+    """absorb_q with q_r rotated by the rotary embedding at positions [T] (int32, device)."""
+    T = q_c.numel() // (dims.num_heads * dims.d_nope)
+    if out is None:
+        out = torch.empty(q_c.shape[:-1] + (dims.d_latent + dims.d_rope,), dtype=torch.bfloat16,
+                          device=q_c.device)
+    assert positions.dtype == torch.int32 and positions.numel() == T
+    _b.check(_b.lib.mla_absorb_q_rope(ctypes.byref(dims), _ptr(q_c), _ptr(q_r), _ptr(w_uk),
+                                      _ptr(positions), float(theta), _ptr(out), T, _stream(stream)),
+             "mla_absorb_q_rope")
+    return out
+
+
 def absorb_out(o_lat, w_uv, dims, out=None, stream=None):
     T = o_lat.numel() // (dims.num_heads * dims.d_latent)
     if out is None:

@@ -154,7 +154,7 @@ mla_status map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, ui
 // out[t, h, :n_cols] = x[t, h, :K] W[h] on tensor cores (+ RoPE copy when rope != null).
 mla_status launch_proj(const void *x, const void *w, void *out, const void *rope, int32_t T,
                        int32_t H, int32_t K, int32_t n_cols, int32_t out_stride, int32_t d_rope,
-                       cudaStream_t s) {
+                       cudaStream_t s, const int32_t *positions = nullptr, double log_theta = 0.0) {
     const int NT = T >= 256 ? 256 : ((T + 15) / 16) * 16;
     CUtensorMap mw, mx;
     mla_status st;
@@ -166,6 +166,8 @@ mla_status launch_proj(const void *x, const void *w, void *out, const void *rope
     mla::ProjArgs a;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.rope = static_cast<const __nv_bfloat16 *>(rope);
+    a.positions = positions;
+    a.log_theta = log_theta;
     a.timeout_ns = kDefaultTimeoutNs;
     a.T = T;
     a.H = H;
@@ -269,6 +271,25 @@ mla_status mla_absorb_q(const mla_dims *dims, const void *q_c, const void *q_r, 
     return launch_proj(q_c, w_uk, q_out, q_r, num_tokens, dims->num_heads, dims->d_nope,
                        dims->d_latent, dims->d_latent + dims->d_rope, dims->d_rope,
                        static_cast<cudaStream_t>(stream));
+}
+
+mla_status mla_absorb_q_rope(const mla_dims *dims, const void *q_c, const void *q_r,
+                             const void *w_uk, const int32_t *positions, float rope_theta,
+                             void *q_out, int32_t num_tokens, void *stream) {
+    mla_status st = check_dims(dims, false);
+    if (st != MLA_OK) return st;
+    if (num_tokens < 0 || !(rope_theta > 1.f) || !std::isfinite(rope_theta)) return MLA_ERR_INVALID_ARG;
+    if (dims->d_nope > 4096 || dims->d_latent > 4096) return MLA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return MLA_OK;
+    if (!q_c || !q_r || !w_uk || !q_out || !positions) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q_c, 16) || !aligned(q_r, 16) || !aligned(w_uk, 16) || !aligned(q_out, 16) ||
+        !aligned(positions, 4))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    return launch_proj(q_c, w_uk, q_out, q_r, num_tokens, dims->num_heads, dims->d_nope,
+                       dims->d_latent, dims->d_latent + dims->d_rope, dims->d_rope,
+                       static_cast<cudaStream_t>(stream), positions,
+                       std::log(static_cast<double>(rope_theta)));
 }
 
 mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w_uv, void *out,

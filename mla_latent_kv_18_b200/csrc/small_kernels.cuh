@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
 struct ProjArgs {
     __nv_bfloat16 *out;          // [T, H, out_stride]
     const __nv_bfloat16 *rope;   // [T, H, d_rope] or null (absorb-in copies q_r)
+    const int32_t *positions;    // [T] or null: rotate the copied q_r (rotary embedding)
+    double log_theta;            // ln(rope_theta) when positions is set
     int64_t timeout_ns;
     int32_t T, H, K, n_cols, out_stride, d_rope, NT;
     int32_t stages;              // ring depth: min(kProjStages, K blocks)
@@ -312,10 +314,35 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
         }
     }
     if (a.rope && blockIdx.y == 0) {
-        for (int i = threadIdx.x; i < nt * a.d_rope; i += 128) {
-            const int t = i / a.d_rope, j = i - t * a.d_rope;
-            a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + a.n_cols + j] =
-                a.rope[(static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + j];
+        // q_r copied pair by pair; with positions, pair (2p, 2p + 1) turns by
+        // pos * theta^(-2p / d_rope) ("MHA2MLA" page §3.2): angle and its
+        // reduction to [-pi, pi] in fp64 (large positions keep their phase),
+        // the rotation itself in fp32, the result rounded to bf16
+        const int half_r = a.d_rope / 2;
+        for (int i = threadIdx.x; i < nt * half_r; i += 128) {
+            const int t = i / half_r, pr = i - t * half_r;
+            const int64_t src = (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + 2 * pr;
+            const int64_t dst = (static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + a.n_cols + 2 * pr;
+            const __nv_bfloat16 x0 = a.rope[src], x1 = a.rope[src + 1];
+            if (a.positions) {
+                int32_t pos = a.positions[t0 + t];
+                if (pos < 0) {
+                    record_error(kErrDeviceBounds);
+                    pos = 0;
+                }
+                const double freq = exp(-2.0 * pr / a.d_rope * a.log_theta);
+                const double ang = static_cast<double>(pos) * freq;
+                const double two_pi = 6.283185307179586476925286766559;
+                double sd, cd;
+                sincos(ang - two_pi * rint(ang / two_pi), &sd, &cd);
+                const float c = static_cast<float>(cd), sn = static_cast<float>(sd);
+                const float f0 = __bfloat162float(x0), f1 = __bfloat162float(x1);
+                a.out[dst] = __float2bfloat16_rn(f0 * c - f1 * sn);
+                a.out[dst + 1] = __float2bfloat16_rn(f0 * sn + f1 * c);
+            } else {
+                a.out[dst] = x0;
+                a.out[dst + 1] = x1;
+            }
         }
     }
     ptx::tc_fence_before();

@@ -309,6 +309,42 @@ def test_fused_combine_absorb_out(api, name, kw):
     assert torch.equal(again, out)
 
 
+@pytest.mark.parametrize("name,kw", [("dsv3", dict(batch=3, heads=16, seq_len=300)),
+                                     ("retrofit", dict(batch=4, seq_len=900))])
+def test_absorb_q_with_rotary_embedding(api, name, kw):
+    """mla_absorb_q_rope: the latent part equals mla_absorb_q's bit for bit, the
+    RoPE part is the oracle's fp64 rotation within one bf16 rounding (large
+    positions included), and position 0 leaves q_r unchanged bit for bit."""
+    w = workload(name, **kw)
+    inp = make_inputs(w, seed=16)
+    d = to_device(inp, "cuda")
+    dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
+    T = w.batch * w.n_q
+    pos = torch.tensor([int(L) - w.n_q + i for L in inp["seq_lens"] for i in range(w.n_q)],
+                       dtype=torch.int32)
+    pos[: min(4, T)] = torch.tensor([0, 1, 65535, 1_000_003][: min(4, T)], dtype=torch.int32)
+    q = api.absorb_q_rope(d["q_c"], d["q_r"], d["w_uk"], dims, pos.cuda())
+    q0 = api.absorb_q(d["q_c"], d["q_r"], d["w_uk"], dims)
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    D = w.d_latent
+    assert torch.equal(q[..., :D], q0[..., :D])
+    ref = oracle.rope(inp["q_r"].reshape(T, w.heads, w.d_rope), pos.numpy())
+    _check_rounded(_f64(q[..., D:]).reshape(ref.shape), ref, "rotated q_r")
+    q_zero = api.absorb_q_rope(d["q_c"], d["q_r"], d["w_uk"], dims, torch.zeros_like(pos).cuda())
+    assert torch.equal(q_zero[..., D:].cpu(), inp["q_r"])
+
+
+def test_absorb_q_rope_negative_position_sets_device_error(api):
+    w = workload("dsv3", batch=2, heads=16, seq_len=300)
+    d = to_device(make_inputs(w, seed=17), "cuda")
+    dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
+    api.absorb_q_rope(d["q_c"], d["q_r"], d["w_uk"], dims,
+                      torch.tensor([5, -3], dtype=torch.int32, device="cuda"))
+    assert api.get_device_error() == 4
+    assert api.get_device_error() == 0
+
+
 def test_repeat_calls_are_bitwise_identical(api):
     w = workload("ragged", batch=8, heads=128, ragged=(500, 5000))
     inp_d = to_device(make_inputs(w, seed=9), "cuda")
