@@ -143,6 +143,25 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(seen), "samples": len(win)}
 
 
+def _max_over_ranks(values, world, device):
+    """Elementwise maximum of a list of floats over all ranks (the job's time is
+    its slowest rank's). Identity for one rank; needs an initialised process
+    group otherwise (nccl with a CUDA device, gloo with "cpu")."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def _job_value(world, tokens_per_step, steps, ms):
+    """Whole-job throughput: every rank processes its own batch (weak scaling),
+    over the slowest rank's time in ms."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def _dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -317,16 +336,9 @@ def main():
     e_ms = e_start.elapsed_time(e_end)
     sampler.stop()
 
-    def allmax(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    ms, e_ms, decode_ms = allmax(ms), allmax(e_ms), allmax(decode_ms)
-    value = world * tokens_per_step * a.steps / (ms / 1e3)
-    e2e_value = world * tokens_per_step * e_steps / (e_ms / 1e3)
+    ms, e_ms, decode_ms = _max_over_ranks([ms, e_ms, decode_ms], world, dev)
+    value = _job_value(world, tokens_per_step, a.steps, ms)
+    e2e_value = _job_value(world, tokens_per_step, e_steps, e_ms)
 
     hbm, tflops, src = _peaks()
     R = w.n_q * w.heads
