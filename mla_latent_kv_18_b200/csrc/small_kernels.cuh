@@ -67,7 +67,21 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
     const int lane = threadIdx.x & 31;
     bool bad = false;
     int64_t N = 0;
-    for (int32_t b0 = 0; b0 < batch; b0 += 32) {
+    constexpr int kCached = 8;   // per-lane tile counts kept for the second pass (batch <= 256)
+    int64_t nc[kCached];
+#pragma unroll
+    for (int c = 0; c < kCached; ++c) {   // all loads of the cached chunks issued together
+        const int32_t bb = 32 * c + lane;
+        nc[c] = (bb < batch) ? tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens) : 0;
+    }
+#pragma unroll
+    for (int c = 0; c < kCached; ++c) {
+        if (32 * c >= batch) break;   // uniform over the warp
+        int64_t n = nc[c];
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        N += n;
+    }
+    for (int32_t b0 = 32 * kCached; b0 < batch; b0 += 32) {
         const int32_t bb = b0 + lane;
         int64_t n = 0;
         if (bb < batch) n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
@@ -84,8 +98,14 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
     for (int32_t b0 = 0; b0 <= b_hi; b0 += 32) {
         const int32_t bb = b0 + lane;
         int64_t n = 0;
-        if (bb < batch && bb <= b_hi)
-            n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        if (bb < batch && bb <= b_hi) {
+            int64_t cached = -1;
+#pragma unroll
+            for (int c = 0; c < kCached; ++c)
+                if (b0 == 32 * c) cached = nc[c];
+            n = cached >= 0 ? cached
+                            : tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        }
         int64_t incl = n;
         for (int o = 1; o < 32; o <<= 1) {
             const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -638,13 +658,31 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
         }
         ptx::cluster_sync();
         const int cw = 128 / KS;   // output columns finished by this CTA
-        for (int idx = threadIdx.x; idx < nt * cw; idx += 128) {
-            const int t = idx / cw, cl = static_cast<int>(q) * cw + (idx - t * cw);
+        const int c4 = cw / 4;     // 4-column groups per token
+        for (int idx = threadIdx.x; idx < nt * c4; idx += 128) {
+            const int t = idx / c4, cl = static_cast<int>(q) * cw + 4 * (idx - t * c4);
             const uint32_t off = part_s + (t * 128u + cl) * 4u;
-            float sum = 0.f;
-            for (int rk = 0; rk < KS; ++rk) sum += ptx::ld_shared_cluster_f32(ptx::mapa(off, rk));
-            if (cl < a.d_v)
-                a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.d_v + cl] = __float2bfloat16_rn(sum);
+            float4 pr[8];   // KS <= 8: every rank's partial requested before any is added
+#pragma unroll
+            for (int rk = 0; rk < 8; ++rk)
+                if (rk < KS) pr[rk] = ptx::ld_shared_cluster_v4(ptx::mapa(off, rk));
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int rk = 0; rk < 8; ++rk)
+                if (rk < KS) {
+                    sum.x += pr[rk].x;
+                    sum.y += pr[rk].y;
+                    sum.z += pr[rk].z;
+                    sum.w += pr[rk].w;
+                }
+            if (cl < a.d_v) {   // d_v is a multiple of 8: the group is all in or all out
+                __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+                uint2 packed;
+                packed.x = *reinterpret_cast<uint32_t *>(&lo);
+                packed.y = *reinterpret_cast<uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(a.out + (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_v + cl) = packed;
+            }
         }
         ptx::cluster_sync();   // peers read this CTA's tile until here
     }
