@@ -205,9 +205,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::mbar_init(bar(&misc->qk_full[i]), 1);
             ptx::mbar_init(bar(&misc->qk_empty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < PV_STAGES; ++i) {
             ptx::mbar_init(bar(&misc->pv_full[i]), 1);
             ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(&misc->s_full[i]), 1);
             ptx::mbar_init(bar(&misc->p_ready[i]), 8);
             ptx::mbar_init(bar(&misc->pv_done[i]), 1);
@@ -372,14 +374,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const bool first = (tp == wp.t_begin);
                     if (first && gp > 0 && !o_free_seen)
                         o_free_seen = ptx::mbar_test_wait(bar(&misc->o_free), (gp - 1) & 1);
-                    const int s = static_cast<int>(kp & 1);
+                    const int s = static_cast<int>(kp & 1);            // P buffer, score buffer
+                    const int ps = static_cast<int>(kp % PV_STAGES);   // P.V operand slot
                     if ((!first || gp == 0 || o_free_seen) &&
-                        ptx::mbar_test_wait(bar(&misc->pv_full[s]), (kp >> 1) & 1) &&
+                        ptx::mbar_test_wait(bar(&misc->pv_full[ps]), (kp / PV_STAGES) & 1) &&
                         ptx::mbar_test_wait(bar(&misc->p_ready[s]), (kp >> 1) & 1)) {
                         ptx::tc_fence_after();
                         const uint64_t a0 = ptx::smem_desc(base + OFF_P + s * P_BYTES, 16, 1024,
                                                            ptx::kSwizzle128B);
-                        const uint64_t b0 = ptx::smem_desc(base + OFF_PV + s * STAGE_PV, TOK * 128,
+                        const uint64_t b0 = ptx::smem_desc(base + OFF_PV + ps * STAGE_PV, TOK * 128,
                                                            1024, ptx::kSwizzle128B);
 #pragma unroll
                         for (int c = 0; c < 2; ++c) {
@@ -390,7 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                                     IDESC_PV, (first && kk == 0) ? 0u : 1u);
                             }
                         }
-                        ptx::mma_commit_pair(bar(&misc->pv_empty[s]), 0x3);
+                        ptx::mma_commit_pair(bar(&misc->pv_empty[ps]), 0x3);
                         ptx::mma_commit_pair(bar(&misc->pv_done[s]), 0x3);
                         ++kp;
                         if (++tp == wp.t_end) {
