@@ -137,7 +137,16 @@ def test_parity_retrofit(api):
 
 
 def test_parity_long_context(api):
-    _parity(api, workload("long"), 48, 2)
+    r, inp = _parity(api, workload("long"), 48, 2)
+    # the fused combine + absorb-out on the same full-size partials (the bench's step)
+    d = to_device(inp, "cuda")
+    lse = torch.empty_like(r["lse"])
+    fused = api.combine_absorb_out(r["ws"], d["seq_lens"], d["block_table"].shape[1], r["dims"],
+                                   r["num_parts"], d["w_uv"], lse_out=lse)
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    assert torch.equal(lse, r["lse"])
+    _check_rounded(_f64(fused), _f64(r["out"]), "long: fused vs unfused")
 
 
 @pytest.mark.parametrize("name,parts", [("dsv3", 7), ("dsv3", 1), ("retrofit", 5), ("ragged", 13)])
