@@ -13,6 +13,9 @@ constants 128 heads, d_hc 128, d_c 512, d_R 64, page_size 64 -- and from the
   ragged    B64 n_q1 H128 L ~ U[1024, 32768], permuted page table
   long      B16 n_q1 H128 L65536,             permuted page table
   retrofit  B32 n_q2 H32  d_n120 d_c64 d_R8 L8192, permuted page table
+  prefill   B8  n_q4096 H128 L4096 (the whole prompt is queried, causal),
+            permuted page table ("MLA operator design" §6: batch 8, prompt
+            4096, above the prefill threshold of 256 query tokens)
 
 Draw recipe (one torch CPU generator per workload, seed 0 by default), in this
 order: seq_lens (ragged only: integers uniform on [1024, 32768]), q_c, q_r,
@@ -58,6 +61,7 @@ WORKLOADS = {
     "ragged": Workload("ragged", 64, 1, 128, 128, 512, 64, 128, 64, ragged=(1024, 32768)),
     "long": Workload("long", 16, 1, 128, 128, 512, 64, 128, 64, seq_len=65536),
     "retrofit": Workload("retrofit", 32, 2, 32, 120, 64, 8, 128, 64, seq_len=8192),
+    "prefill": Workload("prefill", 8, 4096, 128, 128, 512, 64, 128, 64, seq_len=4096),
 }
 
 

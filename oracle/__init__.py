@@ -14,6 +14,12 @@ What it computes (page title, section):
   * ``combine`` -- log-sum-exp merge of partial results over disjoint windows.
   * ``absorb_out`` -- o_lat W_UV per head ("MHA2MLA" §2.1, v = c_kv W_uv).
   * ``decode_absorbed`` -- absorb_q -> attend_latent -> absorb_out, all fp64.
+  * ``decompress_kv`` -- K_nope = c_KV W_UK and V = c_KV W_UV per head, for
+    every cached token (the decompress branch, "MLA operator design" §3, §4).
+  * ``prefill_decompress`` -- M causal queries per sequence through the
+    decompress branch: decompress once per (sequence, head), then softmax over
+    the visible tokens, with the natural-log log-sum-exp ("MLA operator design"
+    §3, §6 prefill threshold; "MHA2MLA" §2.1).
   * ``gather`` -- the page-table gather, on raw bf16 bits.
   * cache-size closed forms ("MLA operator design" §1, "MHA2MLA" §4.2).
 
@@ -48,8 +54,13 @@ def _load():
         lib.oracle_absorb_out.argtypes = [i32, i32, i32, i32, P, P, P, P]
         lib.oracle_rope.argtypes = [i32, i32, i32, P, P, ctypes.c_double, P]
         lib.oracle_rope.restype = i32
+        lib.oracle_decompress_kv.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, P, i32, P, P,
+                                             P, i32, P, P]
+        lib.oracle_prefill_decompress.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, f64,
+                                                  P, P, P, P, i32, P, i32, P, P, P, P, i64, P, P]
         for name in ("oracle_gather", "oracle_decode_decompress", "oracle_absorb_q",
-                     "oracle_attend_latent", "oracle_combine", "oracle_absorb_out"):
+                     "oracle_attend_latent", "oracle_combine", "oracle_absorb_out",
+                     "oracle_decompress_kv", "oracle_prefill_decompress"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -159,6 +170,53 @@ def decode_decompress(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, 
                                           _p(wuk), _p(wuv), _p(s), n_sel, _p(out))
     _check(rc, "decode_decompress")
     return out
+
+
+def decompress_kv(ckv_pool, block_table, seq_lens, w_uk, w_uv, max_len=None):
+    """K_nope [B, H, max_len, d_n] and V [B, H, max_len, d_v] in fp64 (rows past
+    each sequence's length are zero)."""
+    ckv = _bits(ckv_pool)
+    num_pages, P, d_c = ckv.shape
+    wuk, wuv = _bits(w_uk), _bits(w_uv)
+    H, d_n, _ = wuk.shape
+    d_v = wuv.shape[-1]
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    B = sl.shape[0]
+    max_len = int(sl.max()) if max_len is None else int(max_len)
+    kn = np.zeros((B, H, max_len, d_n), dtype=np.float64)
+    v = np.zeros((B, H, max_len, d_v), dtype=np.float64)
+    rc = _load().oracle_decompress_kv(B, H, d_n, d_c, d_v, P, _p(ckv), num_pages, _p(bt),
+                                      bt.shape[1], _p(sl), _p(wuk), _p(wuv), max_len, _p(kn), _p(v))
+    _check(rc, "decompress_kv")
+    return kn, v
+
+
+def prefill_decompress(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv,
+                       scale=None, sel=None):
+    """Causal prefill through the decompress branch, fp64.
+
+    q_c [B, M, H, d_n], q_r [B, M, H, d_r]: the last M tokens of each sequence.
+    Returns (out [B, M, H, d_v], lse [B, M, H]); with sel, entries not selected
+    are out = 0, lse = nan.
+    """
+    qc, qr = _bits(q_c), _bits(q_r)
+    B, M, H, d_n = qc.shape
+    d_r = qr.shape[-1]
+    ckv, kr = _bits(ckv_pool), _bits(kr_pool)
+    num_pages, P, d_c = ckv.shape
+    wuk, wuv = _bits(w_uk), _bits(w_uv)
+    d_v = wuv.shape[-1]
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    scale = default_scale(d_n, d_r) if scale is None else scale
+    s, n_sel = _sel(sel)
+    out = np.zeros((B, M, H, d_v), dtype=np.float64)
+    lse = np.full((B, M, H), np.nan, dtype=np.float64)
+    rc = _load().oracle_prefill_decompress(B, M, H, d_n, d_c, d_r, d_v, P, scale, _p(qc),
+                                           _p(qr), _p(ckv), _p(kr), num_pages, _p(bt),
+                                           bt.shape[1], _p(sl), _p(wuk), _p(wuv), _p(s), n_sel,
+                                           _p(out), _p(lse))
+    _check(rc, "prefill_decompress")
+    return out, lse
 
 
 def absorb_q(q_c, w_uk):

@@ -349,3 +349,146 @@ int oracle_absorb_out(int T, int H, int d_c, int d_v, const uint16_t *o_bf16, co
     }
     return 0;
 }
+
+/*
+ * Decompression of the latent cache, path A of the "MLA operator design" page
+ * §4 ("MHA2MLA" page §2.1: k_nope = c_kv W_uk, v = c_kv W_uv), per sequence b,
+ * head h and cached token t < L_b:
+ *   K_nope[b][h][t][d] = sum_c c_KV[t][c] * W_UK[h][d][c]
+ *   V[b][h][t][e]      = sum_c c_KV[t][c] * W_UV[h][c][e]
+ * k_nope [B,H,max_len,d_n] fp64, v [B,H,max_len,d_v] fp64; rows t >= L_b are
+ * left untouched. Either output may be NULL.
+ */
+int oracle_decompress_kv(int B, int H, int d_n, int d_c, int d_v, int P, const uint16_t *ckv,
+                         int num_pages, const int32_t *block_table, int max_pages,
+                         const int32_t *seq_lens, const uint16_t *w_uk, const uint16_t *w_uv,
+                         int max_len, double *k_nope, double *v) {
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] < 0 || seq_lens[b] > max_len ||
+            (int64_t)seq_lens[b] > (int64_t)max_pages * P) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        int b = (int)(bh / H), h = (int)(bh % H);
+        for (int t = 0; t < seq_lens[b]; ++t) {
+            int64_t row = pool_row(block_table, max_pages, P, num_pages, b, t);
+            if (row < 0) { bad = 1; continue; }
+            const uint16_t *c = ckv + row * d_c;
+            if (k_nope) {
+                double *k = k_nope + (bh * max_len + t) * d_n;
+                for (int d = 0; d < d_n; ++d) {
+                    const uint16_t *w = w_uk + ((int64_t)h * d_n + d) * d_c;
+                    double acc = 0.0;
+                    for (int cc = 0; cc < d_c; ++cc) acc += bf16_to_f64(c[cc]) * bf16_to_f64(w[cc]);
+                    k[d] = acc;
+                }
+            }
+            if (v) {
+                double *vv = v + (bh * max_len + t) * d_v;
+                for (int e = 0; e < d_v; ++e) vv[e] = 0.0;
+                for (int cc = 0; cc < d_c; ++cc) {
+                    double cv = bf16_to_f64(c[cc]);
+                    const uint16_t *w = w_uv + ((int64_t)h * d_c + cc) * d_v;
+                    for (int e = 0; e < d_v; ++e) vv[e] += cv * bf16_to_f64(w[e]);
+                }
+            }
+        }
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Prefill through the decompress branch (the "MLA operator design" page §3 and
+ * §6: a query count M at or above the prefill threshold takes path A, decode
+ * takes path B). The M queries of sequence b are its last M tokens: query i sits
+ * at position L_b - M + i and sees tokens t <= L_b - M + i (causal). For each
+ * (b, h), K_nope and V are decompressed once (as in oracle_decompress_kv), then
+ * per query:
+ *   s[t] = scale * (sum_d q_c[d] K_nope[t][d] + sum_j q_r[j] k_R[t][j])
+ *   out[e] = sum_t softmax(s)[t] V[t][e],   lse = m + log(sum_t exp(s[t] - m))
+ * q_c [B,M,H,d_n], q_r [B,M,H,d_r], out [B,M,H,d_v] fp64, lse [B,M,H] fp64.
+ * sel: optional flat (b*M + i)*H + h indices (n_sel of them); only those
+ * outputs are written, and only the (b, h) pairs they touch are decompressed.
+ */
+int oracle_prefill_decompress(int B, int M, int H, int d_n, int d_c, int d_r, int d_v, int P,
+                              double scale, const uint16_t *q_c, const uint16_t *q_r,
+                              const uint16_t *ckv, const uint16_t *kr, int num_pages,
+                              const int32_t *block_table, int max_pages, const int32_t *seq_lens,
+                              const uint16_t *w_uk, const uint16_t *w_uv, const int64_t *sel,
+                              int64_t n_sel, double *out, double *lse) {
+    if (M < 1 || check_lengths(seq_lens, B, M, max_pages, P)) return -1;
+    /* which queries of which (b, h) to compute */
+    char *want = (char *)calloc((size_t)B * M * H, 1);
+    if (!want) return -1;
+    if (sel) {
+        for (int64_t u = 0; u < n_sel; ++u) {
+            if (sel[u] < 0 || sel[u] >= (int64_t)B * M * H) { free(want); return -1; }
+            want[sel[u]] = 1;
+        }
+    } else {
+        memset(want, 1, (size_t)B * M * H);
+    }
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        int b = (int)(bh / H), h = (int)(bh % H);
+        int any = 0;
+        for (int i = 0; i < M && !any; ++i) any = want[((int64_t)b * M + i) * H + h];
+        if (!any) continue;
+        int L = seq_lens[b];
+        double *kn = (double *)malloc(sizeof(double) * (size_t)L * d_n);
+        double *vv = (double *)malloc(sizeof(double) * (size_t)L * d_v);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L);
+        /* decompress this head's keys and values once */
+        for (int t = 0; t < L; ++t) {
+            int64_t row = pool_row(block_table, max_pages, P, num_pages, b, t);
+            if (row < 0) { bad = 1; row = 0; }
+            const uint16_t *c = ckv + row * d_c;
+            for (int d = 0; d < d_n; ++d) {
+                const uint16_t *w = w_uk + ((int64_t)h * d_n + d) * d_c;
+                double acc = 0.0;
+                for (int cc = 0; cc < d_c; ++cc) acc += bf16_to_f64(c[cc]) * bf16_to_f64(w[cc]);
+                kn[(int64_t)t * d_n + d] = acc;
+            }
+            double *vt = vv + (int64_t)t * d_v;
+            for (int e = 0; e < d_v; ++e) vt[e] = 0.0;
+            for (int cc = 0; cc < d_c; ++cc) {
+                double cv = bf16_to_f64(c[cc]);
+                const uint16_t *w = w_uv + ((int64_t)h * d_c + cc) * d_v;
+                for (int e = 0; e < d_v; ++e) vt[e] += cv * bf16_to_f64(w[e]);
+            }
+        }
+        for (int i = 0; i < M; ++i) {
+            int64_t flat = ((int64_t)b * M + i) * H + h;
+            if (!want[flat]) continue;
+            int nvis = L - M + i + 1;
+            const uint16_t *qc = q_c + flat * d_n;
+            const uint16_t *qr = q_r + flat * d_r;
+            double m = -INFINITY;
+            for (int t = 0; t < nvis; ++t) {
+                int64_t row = pool_row(block_table, max_pages, P, num_pages, b, t);
+                if (row < 0) row = 0;
+                const uint16_t *r = kr + row * d_r;
+                double dot = 0.0;
+                for (int d = 0; d < d_n; ++d) dot += bf16_to_f64(qc[d]) * kn[(int64_t)t * d_n + d];
+                for (int j = 0; j < d_r; ++j) dot += bf16_to_f64(qr[j]) * bf16_to_f64(r[j]);
+                s[t] = scale * dot;
+                if (s[t] > m) m = s[t];
+            }
+            double z = 0.0;
+            for (int t = 0; t < nvis; ++t) { s[t] = exp(s[t] - m); z += s[t]; }
+            double *o = out + flat * d_v;
+            for (int e = 0; e < d_v; ++e) o[e] = 0.0;
+            for (int t = 0; t < nvis; ++t) {
+                double p = s[t] / z;
+                for (int e = 0; e < d_v; ++e) o[e] += p * vv[(int64_t)t * d_v + e];
+            }
+            lse[flat] = m + log(z);
+        }
+        free(kn);
+        free(vv);
+        free(s);
+    }
+    free(want);
+    return bad ? -1 : 0;
+}

@@ -504,3 +504,122 @@ def test_rope_scores_depend_only_on_relative_position(d_r):
     # and it is not symmetric in p and q: the angle has a direction
     ra, rb = oracle.rope(x[:2], [p, q]), oracle.rope(z[:2], [q, p])
     assert abs(float(np.dot(ra[0, 0], rb[0, 0])) - float(np.dot(ra[1, 0], rb[1, 0]))) > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# decompress branch (prefill): K_nope / V decompression and causal M x L
+# ---------------------------------------------------------------------------
+
+def test_decompress_kv_orientation_and_brute_force():
+    rng = np.random.default_rng(5)
+    w = workload("ragged", batch=2, heads=3, d_nope=48, d_latent=64, d_v=40, ragged=(70, 130))
+    inp = make_inputs(w, seed=6)
+    W, perms = _onehot_weights(w.heads, w.d_nope, w.d_latent, rng)
+    Wv, permv = _onehot_weights(w.heads, w.d_v, w.d_latent, rng)
+    wuv = _bf16(np.transpose(Wv, (0, 2, 1)))                 # [H, d_c, d_v]: V[t][e] = c[perm(e)]
+    kn, v = oracle.decompress_kv(inp["ckv_pool"], inp["block_table"], inp["seq_lens"], _bf16(W),
+                                 wuv)
+    for b, (c, _) in enumerate(_dense_cache(inp)):
+        L = c.shape[0]
+        for h in range(w.heads):
+            np.testing.assert_array_equal(kn[b, h, :L], c[:, perms[h]])
+            np.testing.assert_array_equal(v[b, h, :L], c[:, permv[h]])
+        assert not kn[b, :, L:].any() and not v[b, :, L:].any()
+    kn, v = oracle.decompress_kv(inp["ckv_pool"], inp["block_table"], inp["seq_lens"],
+                                 inp["w_uk"], inp["w_uv"])
+    for b, (c, _) in enumerate(_dense_cache(inp)):
+        L = c.shape[0]
+        np.testing.assert_allclose(kn[b, :, :L], np.einsum("sc,hdc->hsd", c, _f64(inp["w_uk"])),
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(v[b, :, :L], np.einsum("sc,hce->hse", c, _f64(inp["w_uv"])),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def _prefill_args(inp):
+    return [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+
+
+@pytest.mark.parametrize("M,lens", [(5, (70, 131)), (64, (64, 100)), (130, (130, 130))])
+def test_prefill_matches_definition_and_brute_force(M, lens):
+    # the decompress-once restatement against the per-output definition (itself pinned
+    # above) and against numpy brute force with scipy's softmax / logsumexp
+    w = workload("dsv3", batch=2, n_q=M, heads=3, d_nope=32, d_latent=64, d_rope=16, d_v=24)
+    inp = make_inputs(w, seed=M, seq_lens=lens)
+    out, lse = oracle.prefill_decompress(*_prefill_args(inp))
+    dec = oracle.decode_decompress(*_prefill_args(inp))
+    np.testing.assert_allclose(out, dec, rtol=1e-12, atol=1e-14)
+    scale = oracle.default_scale(w.d_nope, w.d_rope)
+    np.testing.assert_allclose(out, _numpy_reference(inp, scale), rtol=1e-10, atol=1e-12)
+    qc, qr = _f64(inp["q_c"]), _f64(inp["q_r"])
+    for b, (c, r) in enumerate(_dense_cache(inp)):
+        L = c.shape[0]
+        k_nope = np.einsum("sc,hdc->shd", c, _f64(inp["w_uk"]))
+        for i in (0, M // 2, M - 1):
+            vis = L - M + i + 1
+            s = (np.einsum("hd,shd->hs", qc[b, i], k_nope[:vis])
+                 + np.einsum("hj,sj->hs", qr[b, i], r[:vis])) * scale
+            np.testing.assert_allclose(lse[b, i], scipy.special.logsumexp(s, axis=-1),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_full_prompt_first_query_returns_first_value():
+    # M = L: query 0 sees token 0 only, so out = c_KV[0] W_UV[h] and lse = its score
+    w = workload("dsv3", batch=2, n_q=70, heads=3, d_nope=32, d_latent=64, d_rope=16, d_v=24)
+    inp = make_inputs(w, seed=3, seq_lens=(70, 70))
+    out, lse = oracle.prefill_decompress(*_prefill_args(inp))
+    scale = oracle.default_scale(w.d_nope, w.d_rope)
+    wuk, wuv = _f64(inp["w_uk"]), _f64(inp["w_uv"])
+    qc, qr = _f64(inp["q_c"]), _f64(inp["q_r"])
+    for b, (c, r) in enumerate(_dense_cache(inp)):
+        np.testing.assert_allclose(out[b, 0], np.einsum("c,hce->he", c[0], wuv), rtol=1e-12,
+                                   atol=1e-14)
+        s0 = (np.einsum("hd,hdc,c->h", qc[b, 0], wuk, c[0]) + qr[b, 0] @ r[0]) * scale
+        np.testing.assert_allclose(lse[b, 0], s0, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_zero_query_gives_prefix_means_and_log_counts():
+    w = workload("dsv3", batch=1, n_q=40, heads=2, d_nope=32, d_latent=64, d_rope=16, d_v=24)
+    inp = make_inputs(w, seed=4, seq_lens=(100,))
+    inp["q_c"] = torch.zeros_like(inp["q_c"])
+    inp["q_r"] = torch.zeros_like(inp["q_r"])
+    out, lse = oracle.prefill_decompress(*_prefill_args(inp))
+    (c, _), = _dense_cache(inp)
+    v = np.einsum("sc,hce->she", c, _f64(inp["w_uv"]))
+    for i in range(40):
+        vis = 100 - 40 + i + 1
+        np.testing.assert_allclose(out[0, i], v[:vis].mean(axis=0), rtol=1e-12, atol=1e-14)
+        assert lse[0, i, 0] == math.log(vis) and lse[0, i, 1] == math.log(vis)
+
+
+def test_prefill_is_causal():
+    # changing the cache at positions > p leaves every query at position <= p unchanged,
+    # and changes the later ones
+    w = workload("dsv3", batch=1, n_q=50, heads=2, d_nope=32, d_latent=64, d_rope=16, d_v=24)
+    inp = make_inputs(w, seed=8, seq_lens=(120,))
+    out, lse = oracle.prefill_decompress(*_prefill_args(inp))
+    p = 95                                       # query index p - (120 - 50) = 25
+    table = inp["block_table"][0]
+    ckv, kr = inp["ckv_pool"].clone(), inp["kr_pool"].clone()
+    for t in range(p + 1, 120):
+        ckv[table[t // 64], t % 64] = -ckv[table[t // 64], t % 64]
+        kr[table[t // 64], t % 64] = 2 * kr[table[t // 64], t % 64]
+    pert = dict(inp, ckv_pool=ckv, kr_pool=kr)
+    out2, lse2 = oracle.prefill_decompress(*_prefill_args(pert))
+    i = p - (120 - 50)
+    np.testing.assert_array_equal(out2[0, :i + 1], out[0, :i + 1])
+    np.testing.assert_array_equal(lse2[0, :i + 1], lse[0, :i + 1])
+    assert np.abs(out2[0, i + 1:] - out[0, i + 1:]).min(axis=-1).max() > 0
+
+
+def test_prefill_sampled_selection_matches_full():
+    w = workload("dsv3", batch=2, n_q=20, heads=3, d_nope=32, d_latent=64, d_rope=16, d_v=24)
+    inp = make_inputs(w, seed=9, seq_lens=(33, 90))
+    out, lse = oracle.prefill_decompress(*_prefill_args(inp))
+    sel = [0, 7, 59, 61, 100, 119]
+    o2, l2 = oracle.prefill_decompress(*_prefill_args(inp), sel=sel)
+    flat_o, flat_l = out.reshape(-1, w.d_v), lse.reshape(-1)
+    np.testing.assert_array_equal(o2.reshape(-1, w.d_v)[sel], flat_o[sel])
+    np.testing.assert_array_equal(l2.reshape(-1)[sel], flat_l[sel])
+    rest = np.setdiff1d(np.arange(flat_l.size), sel)
+    assert not o2.reshape(-1, w.d_v)[rest].any() and np.isnan(l2.reshape(-1)[rest]).all()
