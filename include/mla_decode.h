@@ -279,6 +279,73 @@ mla_status mla_debug_gather(const mla_pool *pool, int32_t width, int32_t num_pag
  */
 mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Prefill through the decompress branch.
+ *
+ * The "MLA operator design" page (§3 constant kPrefillThresh, §6 threshold
+ * sweep) routes a step by its query count M: M >= MLA_PREFILL_THRESHOLD takes
+ * the decompress path (path A of §4: K_nope = c_KV W_UK[h]^T and
+ * V = c_KV W_UV[h] per head, "MHA2MLA" page §2.1), below it the absorbed
+ * decode path above. With many queries the per-head widths (d_n + d_R = 192,
+ * d_v = 128) cost fewer FLOPs per (query, key, head) than the latent ones
+ * (576, 512). Compiled specialisation: d_latent 512, d_rope 64, d_nope 128,
+ * d_v 128, page_size 64 (MLA_ERR_UNSUPPORTED otherwise). dims->n_q is M.
+ * The M queries of sequence b are its last M tokens: query i sits at position
+ * seq_lens[b] - M + i and sees tokens t <= seq_lens[b] - M + i (causal).
+ * ------------------------------------------------------------------------ */
+#define MLA_PREFILL_THRESHOLD 256
+
+/* Bytes of the decompressed-cache workspace for `batch` sequences of at most
+ * max_pages_per_seq pages. Layout, with Lpad = max_pages_per_seq * 64 rounded
+ * up to a multiple of 128 and half = align256(batch * H * Lpad * 128 * 2):
+ *   offset 0:     K_nope [batch, H, Lpad, 128] bf16
+ *   offset half:  V      [batch, H, Lpad, 128] bf16
+ * Returns 0 for unsupported dims or bad sizes. */
+size_t mla_prefill_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t max_pages_per_seq);
+
+/*
+ * Decompression ("MHA2MLA" §2.1): for every sequence b, head h and token
+ * t < round_up(seq_lens[b], 128),
+ *   K_nope[b, h, t, d] = bf16( sum_c c_KV[t, c] W_UK[h, d, c] )
+ *   V[b, h, t, e]      = bf16( sum_c c_KV[t, c] W_UV[h, c, e] )
+ * with fp32 accumulation; rows t >= seq_lens[b] are written as zeros. Rows at
+ * or past round_up(seq_lens[b], 128) are not written.
+ * w_uk [H, 128, 512], w_uv [H, 512, 128] bf16 (16-byte aligned); the pool and
+ * table as for mla_decode_splitkv; workspace 256-byte aligned, at least
+ * mla_prefill_workspace_bytes. A page id outside [0, num_pages) or a length
+ * outside [0, max_pages_per_seq * 64] sets MLA_ERR_DEVICE_BOUNDS.
+ */
+mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t num_pages,
+                             const int32_t *block_table, int32_t max_pages_per_seq,
+                             const int32_t *seq_lens, int32_t batch, const void *w_uk,
+                             const void *w_uv, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/*
+ * Causal attention over the decompressed cache written by mla_decompress_kv
+ * (same dims, table, lengths and workspace), for query i of sequence b and
+ * head h:
+ *   s[t]   = scale * (q_c[b, i, h, :] . K_nope[b, h, t, :] + q_r[b, i, h, :] . k_R[t, :])
+ *   out[b, i, h, :] = bf16( sum_t softmax(s)_t V[b, h, t, :] ),  t <= seq_lens[b] - M + i
+ *   lse[b, i, h]    = log sum_t exp(s[t])            (natural log; lse may be NULL)
+ * q_c [batch, M, H, 128], q_r [batch, M, H, 64] bf16 (q_r already rotated, as
+ * the cached k_R is); out [batch, M, H, 128] bf16; lse [batch, M, H] fp32.
+ * scale = dims->softmax_scale, or 1/sqrt(d_nope + d_rope) when <= 0. A length
+ * below M or beyond the table sets MLA_ERR_DEVICE_BOUNDS.
+ */
+mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
+                                 const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                                 const void *workspace, size_t workspace_bytes, void *out,
+                                 float *lse, void *stream);
+
+/* mla_decompress_kv followed by mla_prefill_attention on the same stream. */
+mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, const mla_pool *ckv,
+                       const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                       int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                       const void *w_uk, const void *w_uv, void *workspace,
+                       size_t workspace_bytes, void *out, float *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

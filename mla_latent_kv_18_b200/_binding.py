@@ -18,7 +18,8 @@ EXPORTS = ("mla_absorb_q", "mla_decode_num_parts", "mla_decode_workspace_bytes",
            "mla_decode_splitkv", "mla_combine", "mla_absorb_out", "mla_get_device_error",
            "mla_status_string", "mla_decode_plan", "mla_debug_wait_timeout",
            "mla_decode_latent_noalloc", "mla_debug_gather", "mla_combine_absorb_out",
-           "mla_absorb_q_rope")
+           "mla_absorb_q_rope", "mla_prefill_workspace_bytes", "mla_decompress_kv",
+           "mla_prefill_attention", "mla_prefill")
 
 
 class MLADims(ctypes.Structure):
@@ -61,6 +62,10 @@ def _load():
         "mla_debug_gather": (i32, [PL, i32, i32, P, i32, P, i32, i32, P, P]),
         "mla_combine_absorb_out": (i32, [D, P, sz, P, i32, i32, i32, P, P, P, P]),
         "mla_absorb_q_rope": (i32, [D, P, P, P, P, ctypes.c_float, P, i32, P]),
+        "mla_prefill_workspace_bytes": (sz, [D, i32, i32]),
+        "mla_decompress_kv": (i32, [D, PL, i32, P, i32, P, i32, P, P, P, sz, P]),
+        "mla_prefill_attention": (i32, [D, P, P, PL, i32, P, i32, P, i32, P, sz, P, P, P]),
+        "mla_prefill": (i32, [D, P, P, PL, PL, i32, P, i32, P, i32, P, P, P, sz, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -7,7 +7,9 @@ every step runs in the library's sm_100a kernels.
     o, lse = combine(ws, seq_lens, parts, ...)             # [B, n_q, H, d_c]
     out = absorb_out(o, w_uv)                              # [B, n_q, H, d_v]
 
-or ``decode(...)`` for all four.
+or ``decode(...)`` for all four. A step with many query tokens per sequence
+(``prefill``) decompresses the cache per head instead; ``attend`` routes a
+step by its query count.
 """
 import ctypes
 
@@ -244,3 +246,104 @@ def decode(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, total
     dec = Decoder(dims, block_table.shape[0], block_table.shape[1], total_tiles, q_c.device)
     out = dec(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, stream=stream)
     return out, dec.o_lat, dec.lse
+
+
+# ----------------------------------------------------------------------------
+# prefill through the decompress branch
+# ----------------------------------------------------------------------------
+
+PREFILL_THRESHOLD = 256   # query tokens per sequence from which the decompress branch is taken
+
+
+def prefill_workspace_bytes(dims, batch, max_pages):
+    n = _b.lib.mla_prefill_workspace_bytes(ctypes.byref(dims), batch, max_pages)
+    if n == 0:
+        raise _b.MLAError(2, "mla_prefill_workspace_bytes")
+    return n
+
+
+def alloc_prefill_workspace(dims, batch, max_pages, device):
+    return torch.empty(prefill_workspace_bytes(dims, batch, max_pages), dtype=torch.uint8,
+                       device=device)
+
+
+def prefill_workspace_views(ws, dims, batch, max_pages):
+    """(K_nope, V) views [B, H, Lpad, 128] of a prefill workspace."""
+    l_pad = (max_pages * 64 + 127) // 128 * 128
+    n = batch * dims.num_heads * l_pad * 128
+    half = (n * 2 + 255) // 256 * 256
+    k = ws[:n * 2].view(torch.bfloat16).view(batch, dims.num_heads, l_pad, 128)
+    v = ws[half:half + n * 2].view(torch.bfloat16).view(batch, dims.num_heads, l_pad, 128)
+    return k, v
+
+
+def decompress_kv(ckv_pool, block_table, seq_lens, w_uk, w_uv, dims, workspace=None,
+                  stream=None):
+    """K_nope = c_KV W_UK^T and V = c_KV W_UV per head into the prefill workspace."""
+    B, max_pages = block_table.shape
+    if workspace is None:
+        workspace = alloc_prefill_workspace(dims, B, max_pages, ckv_pool.device)
+    _b.check(_b.lib.mla_decompress_kv(ctypes.byref(dims), ctypes.byref(_pool(ckv_pool)),
+                                      ckv_pool.shape[0], _ptr(block_table), max_pages,
+                                      _ptr(seq_lens), B, _ptr(w_uk), _ptr(w_uv), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "mla_decompress_kv")
+    return workspace
+
+
+def prefill_attention(q_c, q_r, kr_pool, block_table, seq_lens, dims, workspace, out=None,
+                      lse=None, stream=None):
+    """Causal attention of the M = q_c.shape[1] last tokens of each sequence over the
+    decompressed cache. Returns (out [B, M, H, 128], lse [B, M, H])."""
+    B, max_pages = block_table.shape
+    M, H = q_c.shape[1], dims.num_heads
+    if out is None:
+        out = torch.empty(B, M, H, dims.d_v, dtype=torch.bfloat16, device=q_c.device)
+    if lse is None:
+        lse = torch.empty(B, M, H, dtype=torch.float32, device=q_c.device)
+    _b.check(_b.lib.mla_prefill_attention(ctypes.byref(dims), _ptr(q_c), _ptr(q_r),
+                                          ctypes.byref(_pool(kr_pool)), kr_pool.shape[0],
+                                          _ptr(block_table), max_pages, _ptr(seq_lens), B,
+                                          _ptr(workspace), workspace.numel(), _ptr(out),
+                                          _ptr(lse), _stream(stream)), "mla_prefill_attention")
+    return out, lse
+
+
+def prefill(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, scale=0.0,
+            workspace=None, out=None, lse=None, stream=None):
+    """Prefill step through the decompress branch (both kernels). Returns (out, lse)."""
+    dims = dims_for(q_c, q_r, w_uk, w_uv, ckv_pool.shape[1], scale)
+    B, max_pages = block_table.shape
+    M, H = q_c.shape[1], dims.num_heads
+    if workspace is None:
+        workspace = alloc_prefill_workspace(dims, B, max_pages, q_c.device)
+    if out is None:
+        out = torch.empty(B, M, H, dims.d_v, dtype=torch.bfloat16, device=q_c.device)
+    if lse is None:
+        lse = torch.empty(B, M, H, dtype=torch.float32, device=q_c.device)
+    _b.check(_b.lib.mla_prefill(ctypes.byref(dims), _ptr(q_c), _ptr(q_r),
+                                ctypes.byref(_pool(ckv_pool)), ctypes.byref(_pool(kr_pool)),
+                                ckv_pool.shape[0], _ptr(block_table), max_pages, _ptr(seq_lens), B,
+                                _ptr(w_uk), _ptr(w_uv), _ptr(workspace), workspace.numel(),
+                                _ptr(out), _ptr(lse), _stream(stream)), "mla_prefill")
+    return out, lse
+
+
+def route(n_q, heads):
+    """Which branch a step with n_q query tokens per sequence takes: "decompress" at or
+    above the prefill threshold, or when the absorbed kernels cannot hold the
+    n_q * heads query rows (more than 128); "absorb" otherwise."""
+    if n_q >= PREFILL_THRESHOLD or n_q * heads > 128:
+        return "decompress"
+    return "absorb"
+
+
+def attend(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, scale=0.0,
+           stream=None):
+    """One attention step over the paged latent cache, routed by query count.
+    Returns (out [B, n_q, H, d_v], lse [B, n_q, H])."""
+    if route(q_c.shape[1], w_uk.shape[0]) == "decompress":
+        return prefill(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv,
+                       scale=scale, stream=stream)
+    out, _, lse = decode(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv,
+                         scale=scale, stream=stream)
+    return out, lse

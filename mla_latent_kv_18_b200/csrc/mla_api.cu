@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "small_kernels.cuh"
+#include "prefill.cuh"
 
 namespace {
 
@@ -86,7 +87,12 @@ mla_status device_ready() {
             cudaFuncSetAttribute(mla::gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  64 * kGatherMaxWidth * 2) != cudaSuccess ||
             cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 mla::co_smem_bytes(128, mla::kCoMaxNT)) != cudaSuccess) {
+                                 mla::co_smem_bytes(128, mla::kCoMaxNT)) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decompress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::dkv::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::prefill_attn_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::pfa::SMEM_BYTES) != cudaSuccess) {
             st.status = MLA_ERR_CUDA;
             return;
         }
@@ -578,6 +584,170 @@ mla_status mla_debug_wait_timeout(int64_t timeout_ns, void *stream) {
     if (st != MLA_OK) return st;
     mla::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
     return launch_status();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Prefill through the decompress branch
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int32_t kDecompressHeadsPerCta = 8;
+
+// The one compiled prefill specialisation: DeepSeek-V2/V3 dims.
+mla_status check_prefill_dims(const mla_dims *d) {
+    mla_status st = check_dims(d, false);
+    if (st != MLA_OK) return st;
+    if (d->d_latent != 512 || d->d_rope != 64 || d->d_nope != 128 || d->d_v != 128 ||
+        d->page_size != 64)
+        return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+int64_t prefill_l_pad(int32_t max_pages) { return round_up(static_cast<int64_t>(max_pages) * 64, 128); }
+
+int64_t prefill_half_bytes(const mla_dims *d, int32_t batch, int32_t max_pages) {
+    return round_up(static_cast<int64_t>(batch) * d->num_heads * prefill_l_pad(max_pages) * 128 * 2,
+                    256);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mla_prefill_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t max_pages_per_seq) {
+    if (check_prefill_dims(dims) != MLA_OK || batch < 0 || max_pages_per_seq <= 0) return 0;
+    return static_cast<size_t>(2 * prefill_half_bytes(dims, batch, max_pages_per_seq));
+}
+
+mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t num_pages,
+                             const int32_t *block_table, int32_t max_pages_per_seq,
+                             const int32_t *seq_lens, int32_t batch, const void *w_uk,
+                             const void *w_uv, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+    mla_status st = check_prefill_dims(dims);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!block_table || !seq_lens || !w_uk || !w_uv || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(w_uk, 16) ||
+        !aligned(w_uv, 16) || !aligned(workspace, 256))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    if (workspace_bytes < mla_prefill_workspace_bytes(dims, batch, max_pages_per_seq))
+        return MLA_ERR_INVALID_ARG;
+    const int64_t l_pad = prefill_l_pad(max_pages_per_seq);
+    const int64_t tiles = l_pad / mla::dkv::TOK;
+    if (static_cast<int64_t>(batch) * tiles > (int64_t(1) << 31) - 1 || l_pad > (int64_t(1) << 30))
+        return MLA_ERR_UNSUPPORTED;
+    if ((st = device_ready()) != MLA_OK) return st;
+    const int32_t H = dims->num_heads;
+    CUtensorMap mc, mk, mv;
+    if ((st = pool_map(&mc, ckv, 512, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+        return st;
+    // W_UK [H, d_n, d_c]: box [128 d x 64 c];  W_UV [H, d_c, d_v]: box [64 c x 64 e]
+    if ((st = map_3d(&mk, w_uk, 512, 128, H, 512 * 2, uint64_t(128) * 512 * 2, 64, 128, 1)) != MLA_OK)
+        return st;
+    if ((st = map_3d(&mv, w_uv, 128, 512, H, 128 * 2, uint64_t(512) * 128 * 2, 64, 64, 1)) != MLA_OK)
+        return st;
+    mla::DecompressArgs a;
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.k_nope = static_cast<__nv_bfloat16 *>(workspace);
+    a.v = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(workspace) +
+                                            prefill_half_bytes(dims, batch, max_pages_per_seq));
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.batch = batch;
+    a.heads = H;
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    a.l_pad = static_cast<int32_t>(l_pad);
+    a.tiles_per_seq = static_cast<int32_t>(tiles);
+    a.heads_per_cta = std::min(kDecompressHeadsPerCta, H);
+    dim3 grid(static_cast<unsigned>(batch * tiles),
+              static_cast<unsigned>((H + a.heads_per_cta - 1) / a.heads_per_cta));
+    mla::decompress_kernel<<<grid, mla::dkv::THREADS, mla::dkv::SMEM_BYTES,
+                             static_cast<cudaStream_t>(stream)>>>(mc, mk, mv, a);
+    return launch_status();
+}
+
+mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
+                                 const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                                 const void *workspace, size_t workspace_bytes, void *out,
+                                 float *lse, void *stream) {
+    mla_status st = check_prefill_dims(dims);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!q_c || !q_r || !block_table || !seq_lens || !workspace || !out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q_c, 16) || !aligned(q_r, 16) || !aligned(block_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(workspace, 256) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    if (workspace_bytes < mla_prefill_workspace_bytes(dims, batch, max_pages_per_seq))
+        return MLA_ERR_INVALID_ARG;
+    const int64_t M = dims->n_q, H = dims->num_heads;
+    const int64_t q_blocks = (M + mla::pfa::ROWS - 1) / mla::pfa::ROWS;
+    if (batch > 65535 || H > 65535 || q_blocks > (int64_t(1) << 31) - 1 ||
+        static_cast<int64_t>(batch) * M > (int64_t(1) << 31) - 1)
+        return MLA_ERR_UNSUPPORTED;
+    if ((st = device_ready()) != MLA_OK) return st;
+    const int64_t l_pad = prefill_l_pad(max_pages_per_seq);
+    const uint64_t BM = static_cast<uint64_t>(batch) * M, BH = static_cast<uint64_t>(batch) * H;
+    CUtensorMap mqc, mqr, mk, mv, mkr;
+    if ((st = map_3d(&mqc, q_c, 128, H, BM, 128 * 2, uint64_t(H) * 128 * 2, 64, 1, 128)) != MLA_OK)
+        return st;
+    if ((st = map_3d(&mqr, q_r, 64, H, BM, 64 * 2, uint64_t(H) * 64 * 2, 64, 1, 128)) != MLA_OK)
+        return st;
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    if ((st = map_3d(&mk, ws, 128, l_pad, BH, 128 * 2, uint64_t(l_pad) * 128 * 2, 64, 128, 1)) !=
+        MLA_OK)
+        return st;
+    if ((st = map_3d(&mv, ws + prefill_half_bytes(dims, batch, max_pages_per_seq), 128, l_pad, BH,
+                     128 * 2, uint64_t(l_pad) * 128 * 2, 64, 128, 1)) != MLA_OK)
+        return st;
+    if ((st = pool_map(&mkr, kr, 64, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+        return st;
+    mla::PrefillArgs a;
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.timeout_ns = kDefaultTimeoutNs;
+    a.batch = batch;
+    a.heads = static_cast<int32_t>(H);
+    a.n_q = static_cast<int32_t>(M);
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    a.l_pad = static_cast<int32_t>(l_pad);
+    a.q_blocks = static_cast<int32_t>(q_blocks);
+    a.scale = scale_of(dims);
+    a.scale_log2 = a.scale * 1.4426950408889634f;
+    dim3 grid(static_cast<unsigned>(q_blocks), static_cast<unsigned>(H), static_cast<unsigned>(batch));
+    mla::prefill_attn_kernel<<<grid, mla::pfa::THREADS, mla::pfa::SMEM_BYTES,
+                               static_cast<cudaStream_t>(stream)>>>(mqc, mqr, mk, mv, mkr, a);
+    return launch_status();
+}
+
+mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, const mla_pool *ckv,
+                       const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                       int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                       const void *w_uk, const void *w_uv, void *workspace,
+                       size_t workspace_bytes, void *out, float *lse, void *stream) {
+    mla_status st = check_prefill_dims(dims);
+    if (st != MLA_OK) return st;
+    if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!q_c || !q_r || !out) return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    if ((st = mla_decompress_kv(dims, ckv, num_pages, block_table, max_pages_per_seq, seq_lens,
+                                batch, w_uk, w_uv, workspace, workspace_bytes, stream)) != MLA_OK)
+        return st;
+    return mla_prefill_attention(dims, q_c, q_r, kr, num_pages, block_table, max_pages_per_seq,
+                                 seq_lens, batch, workspace, workspace_bytes, out, lse, stream);
 }
 
 }  // extern "C"
