@@ -2,7 +2,7 @@
 """Benchmark: MLA decode over a paged latent cache on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload long|dsv3|ragged|retrofit|tiny]
+                    [--workload long|dsv3|ragged|retrofit|tiny|prefill]
 
 A step is one pass of the whole decode path -- absorb-in, split-KV decode, and
 the log-sum-exp combine fused with absorb-out (mla_combine_absorb_out; with
@@ -12,6 +12,10 @@ page_size 64, shuffled page table). Inputs (1.2 GB of latent cache) exceed the
 126 MB L2, so no flush is needed between steps. With N GPUs each rank runs its
 own replica (no collective on the data path; weak scaling) and the time is the
 maximum over ranks. One JSON line is printed by rank 0.
+
+--workload prefill times the decompress branch instead: a step is one prefill
+of batch 8 x 4096 prompt tokens (decompression of K_nope / V, then causal
+attention), reported as query tokens/s against the bf16 tensor roofline.
 
 --impl reference times the fp64 CPU oracle on the host cores instead (each
 step a bounded sample of the same workload) and prints the same line with
@@ -32,6 +36,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MLA decode KV-tokens/s per B200 (bf16) + % of HBM/tensor roofline vs CPU oracle"
 UNIT = "KV-tokens/s"
+PREFILL_METRIC = "MLA prefill (decompress branch) query tokens/s per B200 (bf16) + % of tensor roofline"
+PREFILL_UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -48,6 +54,8 @@ def _args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="run combine and absorb-out as two calls instead of the fused one")
@@ -63,6 +71,17 @@ def _peaks():
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+
+
+def _sustained_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
 def _src_hash():
@@ -169,6 +188,45 @@ def _dist_init():
     return world, rank, local
 
 
+def _prefill_flops(w, lens):
+    """Algorithmic FLOPs of one prefill: decompression (two [L x d_c] x [d_c x 128]
+    products per head) and causal attention (192-wide scores, 128-wide values over
+    the visible keys only)."""
+    dk = 2.0 * float(sum(int(L) for L in lens)) * w.d_latent * w.heads * (w.d_nope + w.d_v)
+    vis = float(sum(int(L) * w.n_q - w.n_q * (w.n_q - 1) // 2 for L in lens))
+    at = 2.0 * w.heads * vis * ((w.d_nope + w.d_rope) + w.d_v)
+    return dk, at
+
+
+def _prefill_oracle_sample(w, inp, seed, queries=None):
+    """The fp64 oracle's decompress branch on one random (sequence, head) pair per
+    host thread (the oracle runs one pair per thread), with all queries of each pair
+    or `queries` random ones. Returns (query-token rate, threads, description)."""
+    import numpy as np
+    import oracle
+    args = [inp[k] for k in ("q_c", "q_r", "ckv_pool", "kr_pool", "block_table", "seq_lens",
+                             "w_uk", "w_uv")]
+    rng = np.random.default_rng(seed)
+    B, M, H = w.batch, w.n_q, w.heads
+    cores = oracle.num_threads()
+    pairs = rng.choice(B * H, size=min(cores, B * H), replace=False)
+    sel = []
+    for ph in pairs:
+        b, h = divmod(int(ph), H)
+        qs = np.arange(M) if queries is None else np.sort(rng.choice(M, size=queries,
+                                                                     replace=False))
+        sel.append((b * M + qs.astype(np.int64)) * H + h)
+    sel = np.concatenate(sel)
+    t0 = time.perf_counter()
+    oracle.prefill_decompress(*args, sel=sel)
+    dt = time.perf_counter() - t0
+    desc = (f"{len(pairs)} random (sequence, head) pairs, one per host thread, "
+            f"{'all %d' % M if queries is None else queries} queries of each, fp64 "
+            f"decompress-branch oracle (decompression of the pair's whole sequence included), "
+            f"{dt:.1f} s; query tokens counted as rows / heads")
+    return len(sel) / H / dt, cores, desc
+
+
 def run_reference(a):
     """Times the fp64 CPU oracle on bounded samples of the workload."""
     world, rank, _ = _dist_init()
@@ -177,7 +235,35 @@ def run_reference(a):
     import numpy as np
     import oracle
     from mla_latent_kv_18_b200.inputs import make_inputs, workload
-    w = workload(a.workload)
+    w = workload(a.workload, **({"batch": a.batch} if a.batch > 0 else {}))
+    if w.name == "prefill":
+        inp = make_inputs(w, seed=0)
+        lens = inp["seq_lens"].numpy()
+        cores = oracle.num_threads()
+        for i in range(a.warmup):
+            _prefill_oracle_sample(w, inp, 100 + i, queries=8)
+        t0 = time.perf_counter()
+        for i in range(a.steps):
+            _prefill_oracle_sample(w, inp, i, queries=8)
+        dt = time.perf_counter() - t0
+        npairs = min(cores, w.batch * w.heads)
+        value = a.steps * npairs * 8 / w.heads / dt
+        line = {"impl": "reference", "metric": PREFILL_METRIC, "value": value,
+                "unit": PREFILL_UNIT, "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+                "ms_per_step": 1e3 * dt / max(1, a.steps), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": _workload_desc(w, lens), "batch": w.batch,
+                           "seq_len": w.seq_len, "heads": w.heads,
+                           "parallelism": "oracle on host cores"},
+                "cpu_baseline": {"value": value, "unit": PREFILL_UNIT, "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"per step: {npairs} random (sequence, head) pairs, 8 "
+                                           "random queries of each, through the fp64 "
+                                           "decompress-branch oracle"},
+                "e2e": {"value": value, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     inp = make_inputs(w, seed=0)
     cores = oracle.num_threads()
     R = w.n_q * w.heads
@@ -260,10 +346,12 @@ def main():
     from mla_latent_kv_18_b200 import api
     from mla_latent_kv_18_b200.inputs import make_inputs, to_device, workload
 
-    w = workload(a.workload)
+    w = workload(a.workload, **({"batch": a.batch} if a.batch > 0 else {}))
     inp = make_inputs(w, seed=rank)
     d = to_device(inp, dev)
     lens = inp["seq_lens"].numpy()
+    if w.name == "prefill":
+        return main_prefill(a, w, inp, d, lens, world, rank, local, dev)
     dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
     T = api.tile_tokens(dims)
     total_tiles = int(sum((int(L) + T - 1) // T for L in lens))
@@ -428,6 +516,158 @@ def main():
             "gpu_launches": (4 if a.unfused else 3) * a.steps}
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, a.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main_prefill(a, w, inp, d, lens, world, rank, local, dev):
+    """One step = one prefill of the workload through the decompress branch:
+    mla_decompress_kv then mla_prefill_attention."""
+    import torch
+    import torch.distributed as dist
+    from mla_latent_kv_18_b200 import api
+    dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
+    B, max_pages = d["block_table"].shape
+    M, H = w.n_q, w.heads
+    ws = api.alloc_prefill_workspace(dims, B, max_pages, dev)
+    out = torch.empty(B, M, H, w.d_v, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, M, H, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    tokens_per_step = float(B * M)
+
+    def step(ev=None, x=None, o=None):
+        x = d if x is None else x
+        o = out if o is None else o
+        if ev is not None:
+            ev[0].record(stream)
+        api.decompress_kv(d["ckv_pool"], x["block_table"], x["seq_lens"], d["w_uk"], d["w_uv"],
+                          dims, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        api.prefill_attention(x["q_c"], x["q_r"], d["kr_pool"], x["block_table"], x["seq_lens"],
+                              dims, ws, out=o, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(local).start()
+    for _ in range(max(3, a.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(a.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    assert api.get_device_error() == 0
+    ms = start.elapsed_time(end)
+    dk_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    at_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    # end to end: q_c, q_r, table and lengths from pinned host memory, the output back
+    # to pinned host memory, double-buffered with the copies on a second stream
+    keys = ("q_c", "q_r", "block_table", "seq_lens")
+    h = {k: inp[k].pin_memory() for k in keys}
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    xbuf = [{k: torch.empty_like(d[k]) for k in keys} for _ in range(2)]
+    obuf = [torch.empty_like(out) for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = h_out[0].numel() * h_out[0].element_size()
+    cstream = torch.cuda.Stream(device=dev)
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(a.steps // 2, 10))
+
+    def load(i):
+        j = i % 2
+        with torch.cuda.stream(cstream):
+            if i >= 2:
+                cstream.wait_event(computed[j])
+            for k in keys:
+                xbuf[j][k].copy_(h[k], non_blocking=True)
+            loaded[j].record(cstream)
+
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    cstream.wait_event(e_start)
+    load(0)
+    for i in range(e_steps):
+        j = i % 2
+        if i + 1 < e_steps:
+            load(i + 1)
+        stream.wait_event(loaded[j])
+        if i >= 2:
+            stream.wait_event(drained[j])
+        step(x=xbuf[j], o=obuf[j])
+        computed[j].record(stream)
+        with torch.cuda.stream(cstream):
+            cstream.wait_event(computed[j])
+            h_out[j].copy_(obuf[j], non_blocking=True)
+            drained[j].record(cstream)
+    stream.wait_stream(cstream)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    assert api.get_device_error() == 0
+    e_ms = e_start.elapsed_time(e_end)
+    ms, e_ms, dk_ms, at_ms = _max_over_ranks([ms, e_ms, dk_ms, at_ms], world, dev)
+    value = _job_value(world, tokens_per_step, a.steps, ms)
+    e2e_value = _job_value(world, tokens_per_step, e_steps, e_ms)
+
+    _, burst, bsrc = _peaks()
+    sust, ssrc = _sustained_tflops()
+    dk_fl, at_fl = _prefill_flops(w, lens)
+    achieved = at_fl / (at_ms / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": sust, "unit": "TFLOP/s",
+            "frac": achieved / sust, "traffic": None, "kernel": "prefill_attn_kernel",
+            "peak_source": (f"{ssrc} (MEASURED_PEAKS.json bf16_tflops_sustained: the kernel "
+                            "runs back to back for seconds)"),
+            "frac_of_burst_peak": achieved / burst,
+            "algorithmic_flops_per_launch": at_fl, "attention_ms_per_launch": at_ms,
+            "decompress_kernel": {"ms_per_launch": dk_ms, "algorithmic_flops_per_launch": dk_fl,
+                                  "achieved_tflops": dk_fl / (dk_ms / 1e3) / 1e12,
+                                  "frac": dk_fl / (dk_ms / 1e3) / 1e12 / sust}}
+    line = {"metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": _workload_desc(w, lens), "batch": B, "seq_len": w.seq_len,
+                       "query_tokens_per_sequence": M, "heads": H,
+                       "step_tflop": (dk_fl + at_fl) / 1e12,
+                       "l2": "inputs larger than L2 (q_c + q_r %.2f GB, decompressed K/V %.2f GB), "
+                             "no flush" % ((d["q_c"].numel() + d["q_r"].numel()) * 2 / 1e9,
+                                           ws.numel() / 1e9),
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "step_calls": ["mla_decompress_kv", "mla_prefill_attention"]},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": PREFILL_UNIT, "h2d_bytes_per_step": h2d,
+                    "copies": "pinned host buffers; inputs and output double-buffered, copies on a "
+                              "second stream overlapping the neighbouring steps' compute",
+                    "d2h_bytes_per_step": d2h},
+            "clocks": sampler.summary(wall0, wall1),
+            "gpu_launches": 2 * a.steps}
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, cores, desc = _prefill_oracle_sample(w, inp, 1)
+        line["cpu_baseline"] = {"value": v, "unit": PREFILL_UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

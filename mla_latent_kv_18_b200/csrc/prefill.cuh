@@ -505,12 +505,21 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
             arrive(&misc->s_free[s]);
 
             const int32_t tok0 = TOK * k;
-            float mx = -INFINITY;
+            if (tok0 + TOK - 1 > pos) {                 // a block on (or past) the diagonal
 #pragma unroll
-            for (int j = 0; j < TOK; ++j) {
-                v[j] = (tok0 + j <= pos) ? v[j] : -INFINITY;
-                mx = fmaxf(mx, v[j]);
+                for (int j = 0; j < TOK; ++j) v[j] = (tok0 + j <= pos) ? v[j] : -INFINITY;
             }
+            // eight independent partial maxima / sums: one warp per SM sub-partition runs
+            // this, so a single 128-long dependent chain would expose its full latency
+            float m8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) m8[q] = v[q];
+#pragma unroll
+            for (int j = 8; j < TOK; j += 8)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], v[j + q]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             float alpha = 1.f;
             if (mx > -INFINITY &&
                 (m_run == -INFINITY || (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
@@ -518,12 +527,15 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
                 m_run = mx;
             }
             const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
-            float psum = 0.f;
+            float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < TOK; ++j) {
-                v[j] = exp2f(fmaf(v[j], args.scale_log2, -mb));
-                psum += v[j];
-            }
+            for (int j = 0; j < TOK; j += 8)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    v[j + q] = exp2f(fmaf(v[j + q], args.scale_log2, -mb));
+                    s8[q] += v[j + q];
+                }
+            const float psum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
             l_run = fmaf(l_run, alpha, psum);
             const bool need = (k > 0) && (alpha != 1.f);
             if (__any_sync(0xffffffffu, need)) {
