@@ -346,6 +346,30 @@ mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, c
                        const void *w_uk, const void *w_uv, void *workspace,
                        size_t workspace_bytes, void *out, float *lse, void *stream);
 
+/*
+ * Cache write ("MLA operator design" page §3: paged latent cache, page_size
+ * 64, RoPE computed in fp32; "MHA2MLA" page §3.2: rope_theta): for each new
+ * token t with sequence b = seq_ids[t] and absolute position p = positions[t],
+ *   c_KV pool [block_table[b][p / 64]][p % 64][:] = ckv_new[t, :]      (bit copy)
+ *   k_R  pool [block_table[b][p / 64]][p % 64][:] = RoPE(kr_new[t, :], p)
+ * RoPE turns channel pair (2i, 2i + 1) by p * rope_theta^(-2i / d_rope), angle
+ * and its reduction in fp64, rotation fp32, result bf16 -- the same arithmetic
+ * as mla_absorb_q_rope's q_r, so cached keys and queries rotate alike. With
+ * rope_theta <= 0, k_R is copied unrotated. ckv_new [T, d_latent] bf16
+ * (16-byte aligned), kr_new [T, d_rope] bf16 (unrotated), seq_ids / positions
+ * [T] int32; pools and table as for mla_decode_splitkv (the c_KV pool needs a
+ * 16-byte aligned base and strides that are multiples of 8 elements). Every
+ * other slot of the pools is left untouched; two tokens aimed at the same slot
+ * leave one of them there. A sequence id outside [0, batch), a position outside
+ * [0, max_pages_per_seq * 64) or a page id outside [0, num_pages) skips that
+ * token and sets MLA_ERR_DEVICE_BOUNDS.
+ */
+mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+                         const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
+                         float rope_theta, const mla_pool *ckv, const mla_pool *kr,
+                         int32_t num_pages, const int32_t *block_table, int32_t max_pages_per_seq,
+                         int32_t batch, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -162,6 +162,20 @@ def absorb_out(o_lat, w_uv, dims, out=None, stream=None):
     return out
 
 
+def append_kv(ckv_new, kr_new, seq_ids, positions, ckv_pool, kr_pool, block_table, dims,
+              theta=10000.0, stream=None):
+    """Write new tokens' c_KV and RoPE-rotated k_R into the paged pools (in place).
+    ckv_new [T, d_c], kr_new [T, d_R] (unrotated) bf16; seq_ids, positions [T] int32.
+    theta <= 0 copies k_R unrotated."""
+    T = ckv_new.shape[0]
+    B, max_pages = block_table.shape
+    _b.check(_b.lib.mla_append_kv(ctypes.byref(dims), _ptr(ckv_new), _ptr(kr_new), _ptr(seq_ids),
+                                  _ptr(positions), T, float(theta), ctypes.byref(_pool(ckv_pool)),
+                                  ctypes.byref(_pool(kr_pool)), ckv_pool.shape[0],
+                                  _ptr(block_table), max_pages, B, _stream(stream)),
+             "mla_append_kv")
+
+
 def get_device_error(stream=None):
     code = ctypes.c_int32(0)
     _b.check(_b.lib.mla_get_device_error(ctypes.byref(code), _stream(stream)),

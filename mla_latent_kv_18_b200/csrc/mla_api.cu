@@ -751,3 +751,52 @@ mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, c
 }
 
 }  // extern "C"
+
+extern "C" {
+
+mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+                         const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
+                         float rope_theta, const mla_pool *ckv, const mla_pool *kr,
+                         int32_t num_pages, const int32_t *block_table, int32_t max_pages_per_seq,
+                         int32_t batch, void *stream) {
+    mla_status st = check_dims(dims, false);
+    if (st != MLA_OK) return st;
+    if (dims->page_size != 64 || (dims->d_rope % 2)) return MLA_ERR_UNSUPPORTED;
+    if (num_tokens < 0 || batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0 ||
+        !std::isfinite(rope_theta))
+        return MLA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MLA_OK;
+    if (!ckv_new || !kr_new || !seq_ids || !positions || !block_table) return MLA_ERR_INVALID_ARG;
+    if (!aligned(ckv_new, 16) || !aligned(kr_new, 2) || !aligned(seq_ids, 4) ||
+        !aligned(positions, 4) || !aligned(block_table, 4))
+        return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    if (!kr || !kr->base || !aligned(kr->base, 2) || kr->token_stride < dims->d_rope ||
+        kr->page_stride < kr->token_stride)
+        return MLA_ERR_INVALID_ARG;
+    if ((st = device_ready()) != MLA_OK) return st;
+    mla::AppendArgs a;
+    a.ckv_new = static_cast<const __nv_bfloat16 *>(ckv_new);
+    a.kr_new = static_cast<const __nv_bfloat16 *>(kr_new);
+    a.seq_ids = seq_ids;
+    a.positions = positions;
+    a.block_table = block_table;
+    a.ckv = static_cast<__nv_bfloat16 *>(const_cast<void *>(ckv->base));
+    a.kr = static_cast<__nv_bfloat16 *>(const_cast<void *>(kr->base));
+    a.ckv_page_stride = ckv->page_stride;
+    a.ckv_token_stride = ckv->token_stride;
+    a.kr_page_stride = kr->page_stride;
+    a.kr_token_stride = kr->token_stride;
+    a.rotate = rope_theta > 0.f ? 1 : 0;
+    a.log_theta = rope_theta > 0.f ? std::log(static_cast<double>(rope_theta)) : 0.0;
+    a.T = num_tokens;
+    a.d_c = dims->d_latent;
+    a.d_r = dims->d_rope;
+    a.batch = batch;
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    mla::append_kv_kernel<<<(num_tokens + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -214,6 +214,25 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
 // K blocks through a 4-stage ring, one thread of warp 1 issues the MMAs, all
 // four warps drain TMEM (lane = output column) and store bf16.
 // ---------------------------------------------------------------------------
+// Rotary embedding of one channel pair (2p, 2p + 1) at position pos: the pair
+// turns by pos * theta^(-2p / d_rope) ("MHA2MLA" page §3.2). The angle and its
+// reduction to [-pi, pi] are fp64 (large positions keep their phase), the
+// rotation itself fp32 ("MLA operator design" page §3: RoPE in fp32), the
+// result rounded to bf16.
+__device__ __forceinline__ void rope_rotate_pair(__nv_bfloat16 x0, __nv_bfloat16 x1, int32_t pos,
+                                                 int pr, int d_rope, double log_theta,
+                                                 __nv_bfloat16 *y0, __nv_bfloat16 *y1) {
+    const double freq = exp(-2.0 * pr / d_rope * log_theta);
+    const double ang = static_cast<double>(pos) * freq;
+    const double two_pi = 6.283185307179586476925286766559;
+    double sd, cd;
+    sincos(ang - two_pi * rint(ang / two_pi), &sd, &cd);
+    const float c = static_cast<float>(cd), sn = static_cast<float>(sd);
+    const float f0 = __bfloat162float(x0), f1 = __bfloat162float(x1);
+    *y0 = __float2bfloat16_rn(f0 * c - f1 * sn);
+    *y1 = __float2bfloat16_rn(f0 * sn + f1 * c);
+}
+
 struct ProjArgs {
     __nv_bfloat16 *out;          // [T, H, out_stride]
     const __nv_bfloat16 *rope;   // [T, H, d_rope] or null (absorb-in copies q_r)
@@ -350,15 +369,7 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
                     record_error(kErrDeviceBounds);
                     pos = 0;
                 }
-                const double freq = exp(-2.0 * pr / a.d_rope * a.log_theta);
-                const double ang = static_cast<double>(pos) * freq;
-                const double two_pi = 6.283185307179586476925286766559;
-                double sd, cd;
-                sincos(ang - two_pi * rint(ang / two_pi), &sd, &cd);
-                const float c = static_cast<float>(cd), sn = static_cast<float>(sd);
-                const float f0 = __bfloat162float(x0), f1 = __bfloat162float(x1);
-                a.out[dst] = __float2bfloat16_rn(f0 * c - f1 * sn);
-                a.out[dst + 1] = __float2bfloat16_rn(f0 * sn + f1 * c);
+                rope_rotate_pair(x0, x1, pos, pr, a.d_rope, a.log_theta, &a.out[dst], &a.out[dst + 1]);
             } else {
                 a.out[dst] = x0;
                 a.out[dst + 1] = x1;
@@ -759,6 +770,63 @@ __global__ void wait_timeout_kernel(int64_t timeout_ns) {
     }
     __syncthreads();
     if (threadIdx.x == 0) wait_bounded(ptx::smem_u32(&b), 0, &abort_flag, timeout_ns);
+}
+
+}  // namespace mla
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Cache write: new tokens' latent c_KV and decoupled RoPE key k_R into the
+// paged pools, with the rotary embedding applied to k_R on the way in
+// ("MLA operator design" page §3: page_size 64, RoPE in fp32; "MHA2MLA" page
+// §3.2: rope_theta). One warp per token: the c_KV row is a 16-byte-vector
+// copy, each lane rotates one channel pair of k_R at a time.
+// ---------------------------------------------------------------------------
+struct AppendArgs {
+    const __nv_bfloat16 *ckv_new;   // [T, d_c]
+    const __nv_bfloat16 *kr_new;    // [T, d_r] (unrotated)
+    const int32_t *seq_ids;         // [T]
+    const int32_t *positions;       // [T]
+    const int32_t *block_table;     // [batch, max_pages]
+    __nv_bfloat16 *ckv;             // pool base
+    __nv_bfloat16 *kr;              // pool base
+    int64_t ckv_page_stride, ckv_token_stride, kr_page_stride, kr_token_stride;   // elements
+    double log_theta;               // ln(rope_theta); rotate only if rotate != 0
+    int32_t T, d_c, d_r, batch, max_pages, num_pages, rotate;
+};
+
+__global__ void __launch_bounds__(256) append_kv_kernel(const AppendArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    const int32_t b = a.seq_ids[t], pos = a.positions[t];
+    bool ok = b >= 0 && b < a.batch && pos >= 0 &&
+              static_cast<int64_t>(pos) < static_cast<int64_t>(a.max_pages) * 64;
+    int32_t page = 0;
+    if (ok) {
+        page = a.block_table[static_cast<int64_t>(b) * a.max_pages + pos / 64];
+        ok = page >= 0 && page < a.num_pages;
+    }
+    if (!ok) {                       // uniform over the warp
+        if (lane == 0) record_error(kErrDeviceBounds);
+        return;
+    }
+    const int slot = pos % 64;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.ckv_new + t * a.d_c);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ckv + page * a.ckv_page_stride + slot * a.ckv_token_stride);
+    for (int i = lane; i < a.d_c / 8; i += 32) dst[i] = src[i];
+    const __nv_bfloat16 *r = a.kr_new + t * a.d_r;
+    __nv_bfloat16 *rd = a.kr + page * a.kr_page_stride + slot * a.kr_token_stride;
+    for (int p = lane; p < a.d_r / 2; p += 32) {
+        if (a.rotate) {
+            rope_rotate_pair(r[2 * p], r[2 * p + 1], pos, p, a.d_r, a.log_theta, &rd[2 * p],
+                             &rd[2 * p + 1]);
+        } else {
+            rd[2 * p] = r[2 * p];
+            rd[2 * p + 1] = r[2 * p + 1];
+        }
+    }
 }
 
 }  // namespace mla
