@@ -21,6 +21,10 @@ What it computes (page title, section):
     the visible tokens, with the natural-log log-sum-exp ("MLA operator design"
     §3, §6 prefill threshold; "MHA2MLA" §2.1).
   * ``gather`` -- the page-table gather, on raw bf16 bits.
+  * ``e4m3_value`` / ``e4m3_encode`` / ``quantize_fp8_rows`` / ``dequant_fp8_rows``
+    -- the low-precision latent cache: OCP E4M3 codes with one fp32 scale per
+    cached token ("MLA operator design" introduction and §5 name a quantised
+    cache gather; the format is the standard E4M3 one).
   * cache-size closed forms ("MLA operator design" §1, "MHA2MLA" §4.2).
 
 Parity status: every function above is pinned by ``tests/test_oracle_pins.py``
@@ -58,6 +62,14 @@ def _load():
                                              P, i32, P, P]
         lib.oracle_prefill_decompress.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, f64,
                                                   P, P, P, P, i32, P, i32, P, P, P, P, i64, P, P]
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_value.restype = f64
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_quantize_fp8_rows.argtypes = [i64, i32, P, P, P]
+        lib.oracle_quantize_fp8_rows.restype = None
+        lib.oracle_dequant_fp8_rows.argtypes = [i64, i32, P, P, P]
+        lib.oracle_dequant_fp8_rows.restype = None
         for name in ("oracle_gather", "oracle_decode_decompress", "oracle_absorb_q",
                      "oracle_attend_latent", "oracle_combine", "oracle_absorb_out",
                      "oracle_decompress_kv", "oracle_prefill_decompress"):
@@ -314,6 +326,47 @@ def decode_absorbed(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_
     o_lat, lse = attend_latent(q, ckv_pool, kr_pool, block_table, seq_lens, scale, sel=sel)
     out = absorb_out(o_lat, w_uv)
     return out, o_lat, lse
+
+
+# ----------------------------------------------------------------------------
+# low-precision latent cache (E4M3 codes, one fp32 scale per row)
+# ----------------------------------------------------------------------------
+
+def e4m3_value(code) -> float:
+    return _load().oracle_e4m3_value(int(code))
+
+
+def e4m3_encode(y) -> int:
+    return int(_load().oracle_e4m3_encode(float(np.float32(y))))
+
+
+def quantize_fp8_rows(x):
+    """x [..., d] bf16 -> (codes uint8 [..., d], scales float32 [...])."""
+    xb = _bits(x)
+    lead, d = xb.shape[:-1], xb.shape[-1]
+    R = int(np.prod(lead)) if lead else 1
+    codes = np.zeros(xb.shape, dtype=np.uint8)
+    scales = np.zeros(lead, dtype=np.float32)
+    _load().oracle_quantize_fp8_rows(R, d, _p(xb), _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequant_fp8_rows(codes, scales):
+    """(codes uint8 [..., d], scales float32 [...]) -> bf16 bit patterns (uint16) [..., d]."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    sc = np.ascontiguousarray(np.asarray(scales, dtype=np.float32))
+    lead, d = c.shape[:-1], c.shape[-1]
+    R = int(np.prod(lead)) if lead else 1
+    out = np.zeros(c.shape, dtype=np.uint16)
+    _load().oracle_dequant_fp8_rows(R, d, _p(c), _p(sc), _p(out))
+    return out
+
+
+def bf16_from_bits(bits):
+    """uint16 bf16 bit patterns -> torch bfloat16 tensor (same shape)."""
+    import torch
+    b = np.ascontiguousarray(np.asarray(bits, dtype=np.uint16))
+    return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
 
 
 # ----------------------------------------------------------------------------

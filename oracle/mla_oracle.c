@@ -492,3 +492,91 @@ int oracle_prefill_decompress(int B, int M, int H, int d_n, int d_c, int d_r, in
     free(want);
     return bad ? -1 : 0;
 }
+
+/*
+ * Low-precision latent cache: fp8 E4M3 codes with one fp32 scale per cached
+ * token (the "MLA operator design" page, introduction and §5, names a
+ * quantised latent-cache gather but not its format; the E4M3 format used here
+ * is the OCP 8-bit floating point one: sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits, subnormals at exponent field 0, S.1111.111 = NaN, no
+ * infinities, largest finite 448).
+ */
+
+/* Value of an E4M3 code (NaN for S.1111.111). */
+double oracle_e4m3_value(uint8_t code) {
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);                 /* m/8 * 2^-6 */
+    else v = ldexp(8.0 + m, e - 10);                      /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to the fp32 value y, ties to even mantissa, magnitudes
+ * above 448 saturated to 448 (finite saturation). y must not be NaN. */
+uint8_t oracle_e4m3_encode(float y) {
+    const int sign = signbit(y) ? 1 : 0;
+    double a = fabs((double)y);
+    if (a >= 448.0) return (uint8_t)((sign << 7) | 0x7E);
+    if (a == 0.0) return (uint8_t)(sign << 7);
+    int e2;
+    frexp(a, &e2);                                         /* a = f * 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;                                        /* a in [2^e, 2^(e+1)) */
+    if (e < -6) e = -6;                                    /* subnormal range */
+    const double q = ldexp(1.0, e - 3);                    /* spacing of codes at this exponent */
+    double n = rint(a / q);                                /* exact quotient, ties to even */
+    double v = n * q;                                      /* <= 448: 448 is a code, 480 needs a >= 464 */
+    int code;
+    if (v < ldexp(1.0, -6)) {
+        code = (int)(v / ldexp(1.0, -9));                  /* subnormal: m in 0..7 */
+    } else {
+        int ev2;
+        frexp(v, &ev2);
+        const int ev = ev2 - 1;
+        code = ((ev + 7) << 3) | (int)(v / ldexp(1.0, ev - 3) - 8.0);
+    }
+    return (uint8_t)((sign << 7) | code);
+}
+
+/* bf16 bits of an fp32 value, round to nearest even (finite inputs). */
+static uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    const uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * Quantisation of rows x[r][0..d) (bf16 bits) to E4M3 with one scale per row,
+ * all in IEEE fp32 (the arithmetic the kernels use, so codes agree bit for bit):
+ *   amax = max |x|;  inv = 448 / amax  and  scale = amax / 448  (1 and 1 if amax = 0)
+ *   code[j] = E4M3(x[j] * inv)
+ */
+void oracle_quantize_fp8_rows(int64_t R, int d, const uint16_t *x, uint8_t *codes, float *scales) {
+    for (int64_t r = 0; r < R; ++r) {
+        const uint16_t *xr = x + r * d;
+        float amax = 0.0f;
+        for (int j = 0; j < d; ++j) {
+            const float v = fabsf((float)bf16_to_f64(xr[j]));
+            if (v > amax) amax = v;
+        }
+        volatile float num = 448.0f;
+        const float inv = amax > 0.0f ? num / amax : 1.0f;
+        scales[r] = amax > 0.0f ? amax / num : 1.0f;
+        for (int j = 0; j < d; ++j) {
+            volatile float y = (float)bf16_to_f64(xr[j]) * inv;
+            codes[r * d + j] = oracle_e4m3_encode(y);
+        }
+    }
+}
+
+/* Dequantisation to bf16 bits: bf16( fp32( value(code) * scale ) ). */
+void oracle_dequant_fp8_rows(int64_t R, int d, const uint8_t *codes, const float *scales,
+                             uint16_t *out) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int j = 0; j < d; ++j) {
+            volatile float v = (float)oracle_e4m3_value(codes[r * d + j]) * scales[r];
+            out[r * d + j] = f32_to_bf16_rne(v);
+        }
+}

@@ -623,3 +623,92 @@ def test_prefill_sampled_selection_matches_full():
     np.testing.assert_array_equal(l2.reshape(-1)[sel], flat_l[sel])
     rest = np.setdiff1d(np.arange(flat_l.size), sel)
     assert not o2.reshape(-1, w.d_v)[rest].any() and np.isnan(l2.reshape(-1)[rest]).all()
+
+
+# ---------------------------------------------------------------------------
+# low-precision latent cache: E4M3 codes (OCP 8-bit float) with a per-row scale
+# ---------------------------------------------------------------------------
+
+def test_e4m3_values_match_the_format_and_a_library_decoder():
+    # landmarks of the format: smallest subnormal 2^-9, smallest normal 2^-6, one,
+    # largest finite 448, the NaN code, negative zero
+    assert oracle.e4m3_value(0x00) == 0.0 and oracle.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9 and oracle.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle.e4m3_value(0x38) == 1.0 and oracle.e4m3_value(0x7E) == 448.0
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+    assert math.copysign(1.0, oracle.e4m3_value(0x80)) == -1.0
+    assert oracle.e4m3_value(0xB8) == -1.0
+    # all 256 codes against torch's float8_e4m3fn decoder
+    lib = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    lib = lib.float().double().numpy()
+    ours = np.array([oracle.e4m3_value(c) for c in range(256)])
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(lib))
+    np.testing.assert_array_equal(ours[~np.isnan(ours)], lib[~np.isnan(lib)])
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates():
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    for c in finite:                                  # every code is a fixed point
+        assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c
+    pos = sorted(oracle.e4m3_value(c) for c in range(0x7F))
+    for lo, hi in zip(pos, pos[1:]):                  # midpoints go to the even mantissa
+        mid = (lo + hi) / 2
+        got = oracle.e4m3_value(oracle.e4m3_encode(mid))
+        even = lo if (oracle.e4m3_encode(lo) & 1) == 0 else hi
+        assert got == even, (lo, hi, got)
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_encode(-500.0) == 0xFE
+    for big in (448.0, 455.0, 464.0, 470.0, 479.9):   # beyond the last code: clamp, never NaN
+        assert oracle.e4m3_encode(big) == 0x7E and oracle.e4m3_encode(-big) == 0xFE
+    assert oracle.e4m3_encode(2.0 ** -11) == 0x00 and oracle.e4m3_encode(-0.0) == 0x80
+    # random fp32 values of every magnitude against torch's conversion (which saturates
+    # only up to 464; beyond it returns NaN, where ours clamps to 448)
+    rng = np.random.default_rng(3)
+    y = (rng.standard_normal(20000) * np.exp2(rng.uniform(-12, 9, 20000))).astype(np.float32)
+    y = y[np.abs(y) < 464]
+    lib = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(v) for v in y], dtype=np.uint8)
+    np.testing.assert_array_equal(ours, lib)
+
+
+def test_fp8_row_quantisation_bounds_and_special_rows():
+    rng = np.random.default_rng(4)
+    x = _bf16(rng.standard_normal((40, 512)) * np.exp2(rng.uniform(-8, 8, (40, 1))))
+    x[3] = 0.0                                         # an all-zero row
+    codes, scales = oracle.quantize_fp8_rows(x)
+    xd = _f64(x)
+    amax = np.abs(xd).max(axis=1)
+    for r in range(40):
+        if amax[r] == 0:
+            assert scales[r] == 1.0 and not codes[r].any()
+            continue
+        assert scales[r] == np.float32(np.float32(amax[r]) / np.float32(448.0))
+        # the largest magnitude lands on +-448 and every element within half a code step
+        j = int(np.argmax(np.abs(xd[r])))
+        assert codes[r, j] & 0x7F == 0x7E
+        vals = np.array([oracle.e4m3_value(c) for c in codes[r]])
+        y = xd[r] * (np.float32(448.0) / np.float32(amax[r]))
+        step = np.exp2(np.maximum(np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6))), -6) - 3)
+        assert (np.abs(vals - y) <= step / 2 * (1 + 1e-6)).all()
+    deq = oracle.dequant_fp8_rows(codes, scales)
+    back = _f64(oracle.bf16_from_bits(deq))
+    live = amax > 0
+    assert not back[~live].any()
+    rel = np.abs(back - xd)[live] / np.maximum(np.abs(xd), amax[:, None] * 2.0 ** -6)[live]
+    assert rel.max() <= 2.0 ** -4 + 2.0 ** -8      # E4M3 half-step plus the bf16 rounding
+
+
+def test_fp8_dequant_with_power_of_two_scale_is_exact():
+    codes = np.arange(256, dtype=np.uint8).reshape(4, 64)
+    codes[codes == 0x7F] = 0x7E
+    codes[codes == 0xFF] = 0xFE
+    scales = np.array([1.0, 0.5, 2.0 ** -7, 16.0], dtype=np.float32)
+    got = _f64(oracle.bf16_from_bits(oracle.dequant_fp8_rows(codes, scales)))
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy() * scales[:, None]
+    np.testing.assert_array_equal(got, lib)
+    # any scale: the fp32 product rounded to bf16 to nearest even, as torch's conversions do
+    rng = np.random.default_rng(6)
+    scales = (rng.uniform(0.5, 2.0, 4) * np.exp2(rng.integers(-20, 4, 4))).astype(np.float32)
+    got = oracle.dequant_fp8_rows(codes, scales)
+    prod = torch.from_numpy(codes).view(torch.float8_e4m3fn).float() * torch.from_numpy(scales)[:, None]
+    lib = prod.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, lib)
