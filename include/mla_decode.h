@@ -370,6 +370,47 @@ mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *
                          int32_t num_pages, const int32_t *block_table, int32_t max_pages_per_seq,
                          int32_t batch, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Low-precision latent cache. The "MLA operator design" page (introduction
+ * and §5) gathers a quantised latent cache with 16-byte vector loads but does
+ * not give the format; this library stores c_KV as fp8 E4M3 codes (the OCP
+ * 8-bit floating-point format: bias 7, 3 mantissa bits, largest finite 448)
+ * with one fp32 scale per cached token, and keeps k_R in bf16:
+ *   codes pool [pages, 64, d_latent] uint8 (mla_pool strides in bytes, base
+ *   and strides multiples of 16), scales [pages, 64] fp32 (dense).
+ * Quantisation of a row x (IEEE fp32 throughout):
+ *   amax = max |x|;  inv = 448 / amax;  code = E4M3_rn_satfinite(x * inv);
+ *   scale = amax / 448          (an all-zero row: codes 0, scale 1)
+ * Dequantisation: bf16_rn( fp32_rn( value(code) * scale ) ).
+ * ------------------------------------------------------------------------ */
+
+/* mla_append_kv writing the E4M3 cache: c_KV rows are quantised as above into
+ * the codes pool and their scale into scales[page * 64 + slot]; k_R as in
+ * mla_append_kv. d_latent must be a multiple of 16. */
+mla_status mla_append_kv_fp8(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+                             const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
+                             float rope_theta, const mla_pool *ckv8, float *scales,
+                             const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                             int32_t max_pages_per_seq, int32_t batch, void *stream);
+
+/* Dequantising gather: out[b, t, :] = dequant(codes of token t of sequence b)
+ * for t < seq_lens[b], bf16 [batch, max_len, width]; other rows untouched.
+ * width: a multiple of 16, at most 4096. Bad page ids or lengths set
+ * MLA_ERR_DEVICE_BOUNDS. */
+mla_status mla_gather_dequant_fp8(const mla_pool *ckv8, const float *scales, int32_t width,
+                                  int32_t num_pages, const int32_t *block_table,
+                                  int32_t max_pages_per_seq, const int32_t *seq_lens,
+                                  int32_t batch, int32_t max_len, void *out, void *stream);
+
+/* mla_decompress_kv reading the E4M3 cache: the c_KV tile is dequantised as
+ * above before the products, so the result equals mla_decompress_kv on the
+ * dequantised bf16 cache. Use mla_prefill_attention afterwards as usual. */
+mla_status mla_decompress_kv_fp8(const mla_dims *dims, const mla_pool *ckv8, const float *scales,
+                                 int32_t num_pages, const int32_t *block_table,
+                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                                 const void *w_uk, const void *w_uv, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

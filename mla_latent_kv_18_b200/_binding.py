@@ -19,7 +19,8 @@ EXPORTS = ("mla_absorb_q", "mla_decode_num_parts", "mla_decode_workspace_bytes",
            "mla_status_string", "mla_decode_plan", "mla_debug_wait_timeout",
            "mla_decode_latent_noalloc", "mla_debug_gather", "mla_combine_absorb_out",
            "mla_absorb_q_rope", "mla_prefill_workspace_bytes", "mla_decompress_kv",
-           "mla_prefill_attention", "mla_prefill", "mla_append_kv")
+           "mla_prefill_attention", "mla_prefill", "mla_append_kv",
+           "mla_append_kv_fp8", "mla_gather_dequant_fp8", "mla_decompress_kv_fp8")
 
 
 class MLADims(ctypes.Structure):
@@ -67,6 +68,10 @@ def _load():
         "mla_prefill_attention": (i32, [D, P, P, PL, i32, P, i32, P, i32, P, sz, P, P, P]),
         "mla_prefill": (i32, [D, P, P, PL, PL, i32, P, i32, P, i32, P, P, P, sz, P, P, P]),
         "mla_append_kv": (i32, [D, P, P, P, P, i32, ctypes.c_float, PL, PL, i32, P, i32, i32, P]),
+        "mla_append_kv_fp8": (i32, [D, P, P, P, P, i32, ctypes.c_float, PL, P, PL, i32, P, i32, i32,
+                                    P]),
+        "mla_gather_dequant_fp8": (i32, [PL, P, i32, i32, P, i32, P, i32, i32, P, P]),
+        "mla_decompress_kv_fp8": (i32, [D, PL, P, i32, P, i32, P, i32, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

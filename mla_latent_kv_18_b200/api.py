@@ -176,6 +176,58 @@ def append_kv(ckv_new, kr_new, seq_ids, positions, ckv_pool, kr_pool, block_tabl
              "mla_append_kv")
 
 
+def _pool8(t):
+    """A [pages, 64, C] uint8 E4M3 code pool -> mla_pool (strides in bytes)."""
+    assert t.dtype == torch.uint8 and t.dim() == 3 and t.stride(2) == 1
+    return _b.MLAPool(t.data_ptr(), t.stride(0), t.stride(1))
+
+
+def alloc_fp8_cache(num_pages, d_latent, device):
+    """(codes [pages, 64, d_latent] uint8, scales [pages, 64] float32), zeroed."""
+    return (torch.zeros(num_pages, 64, d_latent, dtype=torch.uint8, device=device),
+            torch.zeros(num_pages, 64, dtype=torch.float32, device=device))
+
+
+def append_kv_fp8(ckv_new, kr_new, seq_ids, positions, ckv8_pool, scales, kr_pool, block_table,
+                  dims, theta=10000.0, stream=None):
+    """As append_kv, quantising c_KV into the E4M3 cache (codes + per-token scales)."""
+    T = ckv_new.shape[0]
+    B, max_pages = block_table.shape
+    _b.check(_b.lib.mla_append_kv_fp8(ctypes.byref(dims), _ptr(ckv_new), _ptr(kr_new),
+                                      _ptr(seq_ids), _ptr(positions), T, float(theta),
+                                      ctypes.byref(_pool8(ckv8_pool)), _ptr(scales),
+                                      ctypes.byref(_pool(kr_pool)), ckv8_pool.shape[0],
+                                      _ptr(block_table), max_pages, B, _stream(stream)),
+             "mla_append_kv_fp8")
+
+
+def gather_dequant_fp8(ckv8_pool, scales, block_table, seq_lens, max_len, out=None, stream=None):
+    """Dense bf16 [B, max_len, d_latent] of the dequantised cache rows (others untouched)."""
+    B, max_pages = block_table.shape
+    width = ckv8_pool.shape[2]
+    if out is None:
+        out = torch.zeros(B, max_len, width, dtype=torch.bfloat16, device=ckv8_pool.device)
+    _b.check(_b.lib.mla_gather_dequant_fp8(ctypes.byref(_pool8(ckv8_pool)), _ptr(scales), width,
+                                           ckv8_pool.shape[0], _ptr(block_table), max_pages,
+                                           _ptr(seq_lens), B, max_len, _ptr(out), _stream(stream)),
+             "mla_gather_dequant_fp8")
+    return out
+
+
+def decompress_kv_fp8(ckv8_pool, scales, block_table, seq_lens, w_uk, w_uv, dims, workspace=None,
+                      stream=None):
+    """decompress_kv reading the E4M3 cache."""
+    B, max_pages = block_table.shape
+    if workspace is None:
+        workspace = alloc_prefill_workspace(dims, B, max_pages, ckv8_pool.device)
+    _b.check(_b.lib.mla_decompress_kv_fp8(ctypes.byref(dims), ctypes.byref(_pool8(ckv8_pool)),
+                                          _ptr(scales), ckv8_pool.shape[0], _ptr(block_table),
+                                          max_pages, _ptr(seq_lens), B, _ptr(w_uk), _ptr(w_uv),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+             "mla_decompress_kv_fp8")
+    return workspace
+
+
 def get_device_error(stream=None):
     code = ctypes.c_int32(0)
     _b.check(_b.lib.mla_get_device_error(ctypes.byref(code), _stream(stream)),

@@ -88,7 +88,11 @@ mla_status device_ready() {
                                  64 * kGatherMaxWidth * 2) != cudaSuccess ||
             cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::co_smem_bytes(128, mla::kCoMaxNT)) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::decompress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(mla::decompress_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::dkv::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decompress_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::dkv::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::prefill_attn_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -621,11 +625,16 @@ size_t mla_prefill_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t 
     return static_cast<size_t>(2 * prefill_half_bytes(dims, batch, max_pages_per_seq));
 }
 
-mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t num_pages,
-                             const int32_t *block_table, int32_t max_pages_per_seq,
-                             const int32_t *seq_lens, int32_t batch, const void *w_uk,
-                             const void *w_uv, void *workspace, size_t workspace_bytes,
-                             void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the bf16 and E4M3 cache forms: ckv (bf16) or ckv8 + scales (E4M3).
+mla_status decompress_common(const mla_dims *dims, const mla_pool *ckv, const mla_pool *ckv8,
+                             const float *scales, int32_t num_pages, const int32_t *block_table,
+                             int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                             const void *w_uk, const void *w_uv, void *workspace,
+                             size_t workspace_bytes, void *stream) {
     mla_status st = check_prefill_dims(dims);
     if (st != MLA_OK) return st;
     if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
@@ -634,7 +643,15 @@ mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t 
     if (!aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(w_uk, 16) ||
         !aligned(w_uv, 16) || !aligned(workspace, 256))
         return MLA_ERR_INVALID_ARG;
-    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    const bool fp8 = ckv8 != nullptr;
+    if (fp8) {
+        if (!ckv8->base || !scales || !aligned(ckv8->base, 16) || !aligned(scales, 4) ||
+            ckv8->token_stride < dims->d_latent || ckv8->page_stride < 64 * ckv8->token_stride ||
+            (ckv8->token_stride % 16) || (ckv8->page_stride % 16))
+            return MLA_ERR_INVALID_ARG;
+    } else if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) {
+        return st;
+    }
     if (workspace_bytes < mla_prefill_workspace_bytes(dims, batch, max_pages_per_seq))
         return MLA_ERR_INVALID_ARG;
     const int64_t l_pad = prefill_l_pad(max_pages_per_seq);
@@ -644,14 +661,22 @@ mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t 
     if ((st = device_ready()) != MLA_OK) return st;
     const int32_t H = dims->num_heads;
     CUtensorMap mc, mk, mv;
-    if ((st = pool_map(&mc, ckv, 512, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-        return st;
     // W_UK [H, d_n, d_c]: box [128 d x 64 c];  W_UV [H, d_c, d_v]: box [64 c x 64 e]
     if ((st = map_3d(&mk, w_uk, 512, 128, H, 512 * 2, uint64_t(128) * 512 * 2, 64, 128, 1)) != MLA_OK)
         return st;
     if ((st = map_3d(&mv, w_uv, 128, 512, H, 128 * 2, uint64_t(512) * 128 * 2, 64, 64, 1)) != MLA_OK)
         return st;
+    if (fp8) {
+        mc = mk;   // unused by the E4M3 form
+    } else if ((st = pool_map(&mc, ckv, 512, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+               MLA_OK) {
+        return st;
+    }
     mla::DecompressArgs a;
+    a.ckv8 = fp8 ? static_cast<const uint8_t *>(ckv8->base) : nullptr;
+    a.scales = scales;
+    a.ckv8_page_stride = fp8 ? ckv8->page_stride : 0;
+    a.ckv8_token_stride = fp8 ? ckv8->token_stride : 0;
     a.block_table = block_table;
     a.seq_lens = seq_lens;
     a.k_nope = static_cast<__nv_bfloat16 *>(workspace);
@@ -667,9 +692,38 @@ mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t 
     a.heads_per_cta = std::min(kDecompressHeadsPerCta, H);
     dim3 grid(static_cast<unsigned>(batch * tiles),
               static_cast<unsigned>((H + a.heads_per_cta - 1) / a.heads_per_cta));
-    mla::decompress_kernel<<<grid, mla::dkv::THREADS, mla::dkv::SMEM_BYTES,
-                             static_cast<cudaStream_t>(stream)>>>(mc, mk, mv, a);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (fp8)
+        mla::decompress_kernel<true><<<grid, mla::dkv::THREADS, mla::dkv::SMEM_BYTES, s>>>(mc, mk, mv, a);
+    else
+        mla::decompress_kernel<false><<<grid, mla::dkv::THREADS, mla::dkv::SMEM_BYTES, s>>>(mc, mk, mv, a);
     return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decompress_kv(const mla_dims *dims, const mla_pool *ckv, int32_t num_pages,
+                             const int32_t *block_table, int32_t max_pages_per_seq,
+                             const int32_t *seq_lens, int32_t batch, const void *w_uk,
+                             const void *w_uv, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+    if (!ckv) return MLA_ERR_INVALID_ARG;
+    return decompress_common(dims, ckv, nullptr, nullptr, num_pages, block_table,
+                             max_pages_per_seq, seq_lens, batch, w_uk, w_uv, workspace,
+                             workspace_bytes, stream);
+}
+
+mla_status mla_decompress_kv_fp8(const mla_dims *dims, const mla_pool *ckv8, const float *scales,
+                                 int32_t num_pages, const int32_t *block_table,
+                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                                 const void *w_uk, const void *w_uv, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    if (!ckv8) return MLA_ERR_INVALID_ARG;
+    return decompress_common(dims, nullptr, ckv8, scales, num_pages, block_table,
+                             max_pages_per_seq, seq_lens, batch, w_uk, w_uv, workspace,
+                             workspace_bytes, stream);
 }
 
 mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
@@ -752,13 +806,14 @@ mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, c
 
 }  // extern "C"
 
-extern "C" {
 
-mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+namespace {
+
+mla_status append_common(const mla_dims *dims, const void *ckv_new, const void *kr_new,
                          const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
-                         float rope_theta, const mla_pool *ckv, const mla_pool *kr,
-                         int32_t num_pages, const int32_t *block_table, int32_t max_pages_per_seq,
-                         int32_t batch, void *stream) {
+                         float rope_theta, const mla_pool *ckv, const mla_pool *ckv8, float *scales,
+                         const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                         int32_t max_pages_per_seq, int32_t batch, void *stream) {
     mla_status st = check_dims(dims, false);
     if (st != MLA_OK) return st;
     if (dims->page_size != 64 || (dims->d_rope % 2)) return MLA_ERR_UNSUPPORTED;
@@ -770,7 +825,16 @@ mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *
     if (!aligned(ckv_new, 16) || !aligned(kr_new, 2) || !aligned(seq_ids, 4) ||
         !aligned(positions, 4) || !aligned(block_table, 4))
         return MLA_ERR_INVALID_ARG;
-    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    const bool fp8 = ckv8 != nullptr;
+    if (fp8) {
+        if (dims->d_latent % 16) return MLA_ERR_UNSUPPORTED;
+        if (!ckv8->base || !scales || !aligned(ckv8->base, 16) || !aligned(scales, 4) ||
+            ckv8->token_stride < dims->d_latent || ckv8->page_stride < 64 * ckv8->token_stride ||
+            (ckv8->token_stride % 16) || (ckv8->page_stride % 16))
+            return MLA_ERR_INVALID_ARG;
+    } else if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) {
+        return st;
+    }
     if (!kr || !kr->base || !aligned(kr->base, 2) || kr->token_stride < dims->d_rope ||
         kr->page_stride < kr->token_stride)
         return MLA_ERR_INVALID_ARG;
@@ -781,10 +845,12 @@ mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *
     a.seq_ids = seq_ids;
     a.positions = positions;
     a.block_table = block_table;
-    a.ckv = static_cast<__nv_bfloat16 *>(const_cast<void *>(ckv->base));
+    a.ckv = fp8 ? nullptr : static_cast<__nv_bfloat16 *>(const_cast<void *>(ckv->base));
+    a.ckv8 = fp8 ? static_cast<uint8_t *>(const_cast<void *>(ckv8->base)) : nullptr;
+    a.scales = scales;
     a.kr = static_cast<__nv_bfloat16 *>(const_cast<void *>(kr->base));
-    a.ckv_page_stride = ckv->page_stride;
-    a.ckv_token_stride = ckv->token_stride;
+    a.ckv_page_stride = fp8 ? ckv8->page_stride : ckv->page_stride;
+    a.ckv_token_stride = fp8 ? ckv8->token_stride : ckv->token_stride;
     a.kr_page_stride = kr->page_stride;
     a.kr_token_stride = kr->token_stride;
     a.rotate = rope_theta > 0.f ? 1 : 0;
@@ -796,6 +862,69 @@ mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *
     a.max_pages = max_pages_per_seq;
     a.num_pages = num_pages;
     mla::append_kv_kernel<<<(num_tokens + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_append_kv(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+                         const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
+                         float rope_theta, const mla_pool *ckv, const mla_pool *kr,
+                         int32_t num_pages, const int32_t *block_table, int32_t max_pages_per_seq,
+                         int32_t batch, void *stream) {
+    if (!ckv) return MLA_ERR_INVALID_ARG;
+    return append_common(dims, ckv_new, kr_new, seq_ids, positions, num_tokens, rope_theta, ckv,
+                         nullptr, nullptr, kr, num_pages, block_table, max_pages_per_seq, batch,
+                         stream);
+}
+
+mla_status mla_append_kv_fp8(const mla_dims *dims, const void *ckv_new, const void *kr_new,
+                             const int32_t *seq_ids, const int32_t *positions, int32_t num_tokens,
+                             float rope_theta, const mla_pool *ckv8, float *scales,
+                             const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                             int32_t max_pages_per_seq, int32_t batch, void *stream) {
+    if (!ckv8) return MLA_ERR_INVALID_ARG;
+    return append_common(dims, ckv_new, kr_new, seq_ids, positions, num_tokens, rope_theta,
+                         nullptr, ckv8, scales, kr, num_pages, block_table, max_pages_per_seq,
+                         batch, stream);
+}
+
+mla_status mla_gather_dequant_fp8(const mla_pool *ckv8, const float *scales, int32_t width,
+                                  int32_t num_pages, const int32_t *block_table,
+                                  int32_t max_pages_per_seq, const int32_t *seq_lens,
+                                  int32_t batch, int32_t max_len, void *out, void *stream) {
+    if (width < 16 || width > 4096 || (width % 16)) return MLA_ERR_UNSUPPORTED;
+    if (!ckv8 || !ckv8->base || !scales || !block_table || !seq_lens || !out)
+        return MLA_ERR_INVALID_ARG;
+    if (batch < 0 || max_len < 0 || max_pages_per_seq <= 0 || num_pages <= 0)
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned(ckv8->base, 16) || !aligned(scales, 4) || !aligned(block_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(out, 16) || ckv8->token_stride < width ||
+        ckv8->page_stride < 64 * ckv8->token_stride || (ckv8->token_stride % 16) ||
+        (ckv8->page_stride % 16))
+        return MLA_ERR_INVALID_ARG;
+    if (batch == 0 || max_len == 0) return MLA_OK;
+    const int64_t rows = static_cast<int64_t>(batch) * max_len;
+    if ((rows + 7) / 8 > (int64_t(1) << 31) - 1) return MLA_ERR_UNSUPPORTED;
+    mla_status st = device_ready();
+    if (st != MLA_OK) return st;
+    mla::GatherFp8Args a;
+    a.ckv8 = static_cast<const uint8_t *>(ckv8->base);
+    a.scales = scales;
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.page_stride = ckv8->page_stride;
+    a.token_stride = ckv8->token_stride;
+    a.width = width;
+    a.num_pages = num_pages;
+    a.max_pages = max_pages_per_seq;
+    a.batch = batch;
+    a.max_len = max_len;
+    mla::gather_dequant_fp8_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0,
+                                     static_cast<cudaStream_t>(stream)>>>(a);
     return launch_status();
 }
 

@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "small_kernels.cuh"
 
 namespace mla {
 
@@ -67,6 +68,9 @@ static_assert(sizeof(Misc) <= MISC_BYTES, "misc");
 }  // namespace dkv
 
 struct DecompressArgs {
+    const uint8_t *ckv8;         // E4M3 cache: pool base (kFp8 only)
+    const float *scales;         // E4M3 cache: [pages, 64] per-token scales (kFp8 only)
+    int64_t ckv8_page_stride, ckv8_token_stride;   // bytes
     const int32_t *block_table;  // [B, max_pages]
     const int32_t *seq_lens;     // [B]
     __nv_bfloat16 *k_nope;       // [B, H, Lpad, 128]
@@ -75,6 +79,11 @@ struct DecompressArgs {
     int32_t batch, heads, max_pages, num_pages, l_pad, tiles_per_seq, heads_per_cta;
 };
 
+// kFp8: the c_KV tile comes from the E4M3 cache; the four epilogue warps
+// dequantise it into the resident shared-memory tile before the first MMA
+// (bf16(value(code) * scale), the cache's dequantisation), so the rest of the
+// kernel is unchanged. map_ckv is unused then.
+template <bool kFp8>
 __global__ void __launch_bounds__(dkv::THREADS, 1)
     decompress_kernel(const __grid_constant__ CUtensorMap map_ckv,
                       const __grid_constant__ CUtensorMap map_wuk,
@@ -102,7 +111,7 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
     if (TOK * tb >= L || nh <= 0) return;          // tile past the sequence: never read
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(bar(&misc->a_full), 1);
+        ptx::mbar_init(bar(&misc->a_full), kFp8 ? 4 : 1);
         for (int i = 0; i < STAGES; ++i) {
             ptx::mbar_init(bar(&misc->w_full[i]), 1);
             ptx::mbar_init(bar(&misc->w_empty[i]), 1);
@@ -127,23 +136,25 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
 
     if (warp == 0) {
         if (ptx::elect_one()) {
-            ptx::prefetch_tensormap(&map_ckv);
+            if (!kFp8) ptx::prefetch_tensormap(&map_ckv);
             ptx::prefetch_tensormap(&map_wuk);
             ptx::prefetch_tensormap(&map_wuv);
-            const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
-            const int32_t npages = (L + 63) / 64;
-            int32_t pg[2] = {trow[2 * tb], (2 * tb + 1 < npages) ? trow[2 * tb + 1] : -1};
-            bool bad = false;
-            if (pg[0] < 0 || pg[0] >= args.num_pages) { bad = true; pg[0] = 0; }
-            if (pg[1] == -1 && !(2 * tb + 1 < npages)) pg[1] = pg[0];   // rows >= L: zeroed on store
-            else if (pg[1] < 0 || pg[1] >= args.num_pages) { bad = true; pg[1] = 0; }
-            if (bad) record_error(kErrDeviceBounds);
             const uint32_t ab = bar(&misc->a_full);
-            ptx::mbar_arrive_expect_tx(ab, A_BYTES);
-            for (int blk = 0; blk < CHUNKS; ++blk)
-                for (int i = 0; i < 2; ++i)
-                    ptx::tma_load_3d(base + OFF_A + blk * (TOK * 128) + i * (64 * 128), &map_ckv, ab,
-                                     64 * blk, 0, pg[i]);
+            if (!kFp8) {
+                const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
+                const int32_t npages = (L + 63) / 64;
+                int32_t pg[2] = {trow[2 * tb], (2 * tb + 1 < npages) ? trow[2 * tb + 1] : -1};
+                bool bad = false;
+                if (pg[0] < 0 || pg[0] >= args.num_pages) { bad = true; pg[0] = 0; }
+                if (pg[1] == -1 && !(2 * tb + 1 < npages)) pg[1] = pg[0];   // rows >= L: zeroed on store
+                else if (pg[1] < 0 || pg[1] >= args.num_pages) { bad = true; pg[1] = 0; }
+                if (bad) record_error(kErrDeviceBounds);
+                ptx::mbar_arrive_expect_tx(ab, A_BYTES);
+                for (int blk = 0; blk < CHUNKS; ++blk)
+                    for (int i = 0; i < 2; ++i)
+                        ptx::tma_load_3d(base + OFF_A + blk * (TOK * 128) + i * (64 * 128), &map_ckv,
+                                         ab, 64 * blk, 0, pg[i]);
+            }
             int n = 0;
             for (; n < total; ++n) {
                 const int st = n % STAGES;
@@ -161,7 +172,7 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
                 ptx::tma_load_3d(sb + WK_BYTES + 64 * 128, &map_wuv, fb, 64, 64 * c, h);
             }
             // no copy may still be landing when the CTA exits (the abort path)
-            wait_bounded<false>(ab, 0, abort_flag, args.timeout_ns);
+            if (!kFp8) wait_bounded<false>(ab, 0, abort_flag, args.timeout_ns);
             for (int m = (n > STAGES ? n - STAGES : 0); m < n; ++m)
                 wait_bounded<false>(bar(&misc->w_full[m % STAGES]), (m / STAGES) & 1, abort_flag,
                                     args.timeout_ns);
@@ -208,6 +219,37 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
             wait_bounded<false>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
         }
     } else {
+        if (kFp8) {
+            // dequantise this warp's 32 tile rows: one 512-byte row per warp load
+            // (16 codes per lane), written as two swizzled 16-byte chunks per lane
+            const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
+            bool bad = false;
+            for (int rr = 0; rr < 32; ++rr) {
+                const int r = 32 * (warp - 2) + rr;
+                const int32_t t = TOK * tb + r;
+                uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                if (t < L) {
+                    const int32_t page = trow[t / 64];
+                    if (page >= 0 && page < args.num_pages) {
+                        const uint8_t *src = args.ckv8 + page * args.ckv8_page_stride +
+                                             (t % 64) * args.ckv8_token_stride;
+                        const float sc = args.scales[static_cast<int64_t>(page) * 64 + (t % 64)];
+                        const uint4 codes = *reinterpret_cast<const uint4 *>(src + 16 * lane);
+                        lo = dequant8_e4m3(codes.x, codes.y, sc);
+                        hi = dequant8_e4m3(codes.z, codes.w, sc);
+                    } else {
+                        bad = true;
+                    }
+                }
+                const uint32_t blk = base + OFF_A + (lane >> 2) * (TOK * 128);
+                st_shared_v4(blk + sw128(r, 2 * (lane & 3)), lo.x, lo.y, lo.z, lo.w);
+                st_shared_v4(blk + sw128(r, 2 * (lane & 3) + 1), hi.x, hi.y, hi.z, hi.w);
+            }
+            if (bad && lane == 0) record_error(kErrDeviceBounds);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(&misc->a_full));
+        }
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int32_t t = TOK * tb + row;

@@ -4,6 +4,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include <cuda.h>
 
@@ -789,7 +790,9 @@ struct AppendArgs {
     const int32_t *seq_ids;         // [T]
     const int32_t *positions;       // [T]
     const int32_t *block_table;     // [batch, max_pages]
-    __nv_bfloat16 *ckv;             // pool base
+    __nv_bfloat16 *ckv;             // pool base (bf16 cache), or null
+    uint8_t *ckv8;                  // pool base (E4M3 cache), or null
+    float *scales;                  // [pages, 64] with the E4M3 cache
     __nv_bfloat16 *kr;              // pool base
     int64_t ckv_page_stride, ckv_token_stride, kr_page_stride, kr_token_stride;   // elements
     double log_theta;               // ln(rope_theta); rotate only if rotate != 0
@@ -814,8 +817,44 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const AppendArgs a) {
     }
     const int slot = pos % 64;
     const uint4 *src = reinterpret_cast<const uint4 *>(a.ckv_new + t * a.d_c);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.ckv + page * a.ckv_page_stride + slot * a.ckv_token_stride);
-    for (int i = lane; i < a.d_c / 8; i += 32) dst[i] = src[i];
+    if (a.ckv8) {
+        // E4M3 with one fp32 scale per token: amax over the row, then
+        // inv = 448 / amax, code = E4M3_rn_satfinite(x * inv), scale = amax / 448,
+        // all with IEEE-rounded fp32 operations
+        float amax = 0.f;
+        for (int i = lane; i < a.d_c / 8; i += 32) {
+            const uint4 v = src[i];
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(h[q]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+        uint8_t *dst8 = a.ckv8 + page * a.ckv_page_stride + slot * a.ckv_token_stride;
+        for (int i = lane; i < a.d_c / 8; i += 32) {
+            const uint4 v = src[i];
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+            uint32_t w[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const float2 f0 = __bfloat1622float2(h[2 * q]), f1 = __bfloat1622float2(h[2 * q + 1]);
+                const uint32_t c0 = __nv_cvt_float_to_fp8(__fmul_rn(f0.x, inv), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t c1 = __nv_cvt_float_to_fp8(__fmul_rn(f0.y, inv), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t c2 = __nv_cvt_float_to_fp8(__fmul_rn(f1.x, inv), __NV_SATFINITE, __NV_E4M3);
+                const uint32_t c3 = __nv_cvt_float_to_fp8(__fmul_rn(f1.y, inv), __NV_SATFINITE, __NV_E4M3);
+                w[q] = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+            }
+            *reinterpret_cast<uint2 *>(dst8 + 8 * i) = make_uint2(w[0], w[1]);
+        }
+        if (lane == 0) a.scales[static_cast<int64_t>(page) * 64 + slot] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(a.ckv + page * a.ckv_page_stride + slot * a.ckv_token_stride);
+        for (int i = lane; i < a.d_c / 8; i += 32) dst[i] = src[i];
+    }
     const __nv_bfloat16 *r = a.kr_new + t * a.d_r;
     __nv_bfloat16 *rd = a.kr + page * a.kr_page_stride + slot * a.kr_token_stride;
     for (int p = lane; p < a.d_r / 2; p += 32) {
@@ -826,6 +865,72 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const AppendArgs a) {
             rd[2 * p] = r[2 * p];
             rd[2 * p + 1] = r[2 * p + 1];
         }
+    }
+}
+
+}  // namespace mla
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Dequantising gather of the E4M3 latent cache (the quantised cache gather of
+// the "MLA operator design" page, introduction and §5, with 16-byte loads):
+//   out[b, t, c] = bf16( value(code[b, t, c]) * scale[b, t] )   for t < seq_lens[b]
+// One warp per (sequence, token) row; each lane loads 16 codes (16 bytes) and
+// writes 32 bytes of bf16.
+// ---------------------------------------------------------------------------
+struct GatherFp8Args {
+    const uint8_t *ckv8;            // pool base
+    const float *scales;            // [pages, 64]
+    const int32_t *block_table;     // [batch, max_pages]
+    const int32_t *seq_lens;        // [batch]
+    __nv_bfloat16 *out;             // [batch, max_len, width]
+    int64_t page_stride, token_stride;   // bytes
+    int32_t width, num_pages, max_pages, batch, max_len;
+};
+
+// 8 E4M3 codes (two 32-bit words, first code in the low byte) to 8 bf16:
+// bf16_rn( fp32_rn( value(code) * scale ) ); value(code) is exact in fp32.
+__device__ __forceinline__ uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float scale) {
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t w = q < 2 ? w0 : w1;
+        const int sh = (q & 1) * 16;
+        __nv_fp8_e4m3 lo, hi;
+        lo.__x = static_cast<__nv_fp8_storage_t>((w >> sh) & 0xFFu);
+        hi.__x = static_cast<__nv_fp8_storage_t>((w >> (sh + 8)) & 0xFFu);
+        const __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(static_cast<float>(lo), scale),
+                                                      __fmul_rn(static_cast<float>(hi), scale));
+        out[q] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__global__ void __launch_bounds__(256) gather_dequant_fp8_kernel(const GatherFp8Args a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= static_cast<int64_t>(a.batch) * a.max_len) return;
+    const int32_t b = static_cast<int32_t>(row / a.max_len);
+    const int32_t t = static_cast<int32_t>(row - static_cast<int64_t>(b) * a.max_len);
+    const int32_t L = a.seq_lens[b];
+    if (L < 0 || L > a.max_len || static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * 64) {
+        if (t == 0 && lane == 0) record_error(kErrDeviceBounds);
+        return;
+    }
+    if (t >= L) return;
+    const int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_pages + t / 64];
+    if (page < 0 || page >= a.num_pages) {
+        if (lane == 0) record_error(kErrDeviceBounds);
+        return;
+    }
+    const uint8_t *src = a.ckv8 + page * a.page_stride + (t % 64) * a.token_stride;
+    const float scale = a.scales[static_cast<int64_t>(page) * 64 + (t % 64)];
+    __nv_bfloat16 *dst = a.out + row * a.width;
+    for (int i = lane; i < a.width / 16; i += 32) {
+        const uint4 codes = *reinterpret_cast<const uint4 *>(src + 16 * i);
+        reinterpret_cast<uint4 *>(dst + 16 * i)[0] = dequant8_e4m3(codes.x, codes.y, scale);
+        reinterpret_cast<uint4 *>(dst + 16 * i)[1] = dequant8_e4m3(codes.z, codes.w, scale);
     }
 }
 
