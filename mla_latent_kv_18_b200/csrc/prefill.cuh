@@ -535,13 +535,15 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
             }
             ptx::tc_fence_after();
             float v[TOK];
+            {
+                uint32_t sr[TOK];
 #pragma unroll
-            for (int c = 0; c < TOK / 32; ++c) {
-                uint32_t sr[32];
-                ptx::tmem_ld32(tmem + lane_base + TMEM_S + TOK * s + 32 * c, sr);
+                for (int c = 0; c < TOK / 32; ++c)
+                    ptx::tmem_ld32(tmem + lane_base + TMEM_S + TOK * s + 32 * c,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[32 * c + j] = __uint_as_float(sr[j]);
+                for (int j = 0; j < TOK; ++j) v[j] = __uint_as_float(sr[j]);
             }
             ptx::tc_fence_before();
             arrive(&misc->s_free[s]);
@@ -628,21 +630,21 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
                 const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
                 __nv_bfloat16 *dst =
                     args.out + ((static_cast<int64_t>(b) * M + i) * args.heads + h) * DV;
-#pragma unroll 1
-                for (int cch = 0; cch < DV / 32; ++cch) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
-                    ptx::tmem_wait_ld();
-                    if (real) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cch);
+                uint32_t o[DV];                         // four loads in flight, one wait
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d4[q] = make_uint4(
-                                pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
-                    }
+                for (int cch = 0; cch < DV / 32; ++cch)
+                    ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&o[32 * cch]));
+                ptx::tmem_wait_ld();
+                if (real) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                    for (int q = 0; q < DV / 8; ++q)
+                        d4[q] = make_uint4(
+                            pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
                 }
                 if (real && args.lse)
                     args.lse[(static_cast<int64_t>(b) * M + i) * args.heads + h] =
