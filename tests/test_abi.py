@@ -146,3 +146,81 @@ def test_argument_validation_without_launch(b):
                                   1, fake, 1, fake, 2, 1, ctypes.c_void_p(0x10010), ws_bytes,
                                   null) == 1                # workspace not 256-byte aligned
     assert lib.mla_debug_wait_timeout(0, null) == 1
+
+
+def test_prefill_workspace_size_and_validation_without_launch(b):
+    lib = b.lib
+    by = ctypes.byref
+    d = _dims(b, n_q=300)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x1000)
+    # K_nope then V, each [B, H, Lpad, 128] bf16 with Lpad = max_pages * 64 rounded up to 128
+    for B, mp in ((2, 5), (8, 64), (1, 1), (3, 2)):
+        l_pad = (mp * 64 + 127) // 128 * 128
+        half = (B * 128 * l_pad * 128 * 2 + 255) // 256 * 256
+        assert lib.mla_prefill_workspace_bytes(by(d), B, mp) == 2 * half
+    # only the DeepSeek specialisation is compiled for the decompress branch
+    dr = _dims(b, d_latent=64, d_rope=8, d_nope=120)
+    assert lib.mla_prefill_workspace_bytes(by(dr), 2, 5) == 0
+    pool = b.MLAPool(0x1000, 64 * 576, 576)
+    kpool = b.MLAPool(0x1000, 64 * 64, 64)
+    args = [fake, fake, by(pool), by(kpool), 4, fake, 2, fake, 2, fake, fake, fake, 1 << 30,
+            fake, null, null]
+    assert lib.mla_prefill(by(dr), *args) == 2
+    assert lib.mla_prefill(by(_dims(b, n_q=300, page_size=16)), *args) == 2
+    # batch 0 is a no-op; null pointers with work to do are rejected
+    a0 = list(args)
+    a0[8] = 0
+    assert lib.mla_prefill(by(d), *a0) == 0
+    a1 = list(args)
+    a1[0] = null
+    assert lib.mla_prefill(by(d), *a1) == 1
+    ws = lib.mla_prefill_workspace_bytes(by(d), 2, 2)
+    assert lib.mla_decompress_kv(by(d), by(pool), 4, fake, 2, fake, 2, fake, fake, fake, ws - 2,
+                                 null) == 1                 # workspace too small
+    assert lib.mla_decompress_kv(by(d), by(pool), 4, fake, 2, fake, 2, fake, fake,
+                                 ctypes.c_void_p(0x1010), ws, null) == 1   # not 256-B aligned
+    assert lib.mla_prefill_attention(by(d), ctypes.c_void_p(0x1002), fake, by(kpool), 4, fake, 2,
+                                     fake, 2, fake, ws, fake, null, null) == 1   # misaligned q_c
+
+
+def test_cache_write_and_fp8_calls_validate_without_launch(b):
+    lib = b.lib
+    by = ctypes.byref
+    d = _dims(b)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x1000)
+    cpool = b.MLAPool(0x1000, 64 * 512, 512)
+    kpool = b.MLAPool(0x1000, 64 * 64, 64)
+    c8 = b.MLAPool(0x1000, 64 * 512, 512)
+    # no tokens: nothing to do; null pointers with tokens: rejected
+    assert lib.mla_append_kv(by(d), null, null, null, null, 0, 10000.0, by(cpool), by(kpool), 4,
+                             null, 2, 2, null) == 0
+    assert lib.mla_append_kv(by(d), null, fake, fake, fake, 3, 10000.0, by(cpool), by(kpool), 4,
+                             fake, 2, 2, null) == 1
+    assert lib.mla_append_kv(by(d), fake, fake, fake, fake, 3, float("nan"), by(cpool), by(kpool),
+                             4, fake, 2, 2, null) == 1      # theta must be finite
+    assert lib.mla_append_kv(by(_dims(b, page_size=32)), fake, fake, fake, fake, 3, 10000.0,
+                             by(cpool), by(kpool), 4, fake, 2, 2, null) == 2   # page size other than 64
+    # the E4M3 cache: latent width a multiple of 16, scales given, 16-byte strides
+    assert lib.mla_append_kv_fp8(by(_dims(b, d_latent=72)), fake, fake, fake, fake, 3, 1e4,
+                                 by(c8), fake, by(kpool), 4, fake, 2, 2, null) == 2
+    assert lib.mla_append_kv_fp8(by(d), fake, fake, fake, fake, 3, 1e4, by(c8), null, by(kpool),
+                                 4, fake, 2, 2, null) == 1
+    odd = b.MLAPool(0x1000, 64 * 520, 520)
+    assert lib.mla_append_kv_fp8(by(d), fake, fake, fake, fake, 3, 1e4, by(odd), fake, by(kpool),
+                                 4, fake, 2, 2, null) == 1
+    # dequantising gather: width, alignment, no-op sizes
+    assert lib.mla_gather_dequant_fp8(by(c8), fake, 24, 4, fake, 2, fake, 2, 10, fake, null) == 2
+    assert lib.mla_gather_dequant_fp8(by(c8), fake, 512, 4, fake, 2, fake, 2, 10,
+                                      ctypes.c_void_p(0x1008), null) == 1
+    assert lib.mla_gather_dequant_fp8(by(c8), fake, 512, 4, fake, 2, fake, 0, 10, fake, null) == 0
+    assert lib.mla_gather_dequant_fp8(by(c8), fake, 512, 4, fake, 2, fake, 2, 0, fake, null) == 0
+    # decompress from the E4M3 cache: scales required, token stride at least the width
+    dp = _dims(b, n_q=300)
+    ws = lib.mla_prefill_workspace_bytes(by(dp), 2, 2)
+    assert lib.mla_decompress_kv_fp8(by(dp), by(c8), null, 4, fake, 2, fake, 2, fake, fake, fake,
+                                     ws, null) == 1
+    short = b.MLAPool(0x1000, 64 * 256, 256)
+    assert lib.mla_decompress_kv_fp8(by(dp), by(short), fake, 4, fake, 2, fake, 2, fake, fake,
+                                     fake, ws, null) == 1
