@@ -656,13 +656,15 @@ mla_status decompress_common(const mla_dims *dims, const mla_pool *ckv, const ml
         return MLA_ERR_INVALID_ARG;
     const int64_t l_pad = prefill_l_pad(max_pages_per_seq);
     const int64_t tiles = l_pad / mla::dkv::TOK;
-    if (static_cast<int64_t>(batch) * tiles > (int64_t(1) << 31) - 1 || l_pad > (int64_t(1) << 30))
+    if (2 * static_cast<int64_t>(batch) * ((tiles + 1) / 2) > (int64_t(1) << 31) - 1 ||
+        l_pad > (int64_t(1) << 30))
         return MLA_ERR_UNSUPPORTED;
     if ((st = device_ready()) != MLA_OK) return st;
     const int32_t H = dims->num_heads;
     CUtensorMap mc, mk, mv;
-    // W_UK [H, d_n, d_c]: box [128 d x 64 c];  W_UV [H, d_c, d_v]: box [64 c x 64 e]
-    if ((st = map_3d(&mk, w_uk, 512, 128, H, 512 * 2, uint64_t(128) * 512 * 2, 64, 128, 1)) != MLA_OK)
+    // W_UK [H, d_n, d_c]: box [64 d x 64 c];  W_UV [H, d_c, d_v]: box [64 c x 64 e] (each CTA
+    // of a pair loads its half of a chunk)
+    if ((st = map_3d(&mk, w_uk, 512, 128, H, 512 * 2, uint64_t(128) * 512 * 2, 64, 64, 1)) != MLA_OK)
         return st;
     if ((st = map_3d(&mv, w_uv, 128, 512, H, 128 * 2, uint64_t(512) * 128 * 2, 64, 64, 1)) != MLA_OK)
         return st;
@@ -688,9 +690,9 @@ mla_status decompress_common(const mla_dims *dims, const mla_pool *ckv, const ml
     a.max_pages = max_pages_per_seq;
     a.num_pages = num_pages;
     a.l_pad = static_cast<int32_t>(l_pad);
-    a.tiles_per_seq = static_cast<int32_t>(tiles);
+    a.pairs_per_seq = static_cast<int32_t>((tiles + 1) / 2);
     a.heads_per_cta = std::min(kDecompressHeadsPerCta, H);
-    dim3 grid(static_cast<unsigned>(batch * tiles),
+    dim3 grid(static_cast<unsigned>(2 * batch * ((tiles + 1) / 2)),   // CTA pairs (clusters of 2)
               static_cast<unsigned>((H + a.heads_per_cta - 1) / a.heads_per_cta));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (fp8)

@@ -36,30 +36,35 @@ namespace mla {
 // decompress_kernel
 // ===========================================================================
 namespace dkv {
-constexpr int TOK = 128;                         // tokens per tile (two pages)
+constexpr int TOK = 128;                         // tokens per CTA tile (two pages)
 constexpr int DC = 512, DN = 128, DV = 128;
 constexpr int CHUNKS = DC / 64;                  // 64-channel K chunks
 constexpr uint32_t A_BYTES = TOK * DC * 2;       // 8 swizzled blocks [128 tok x 64 ch]
-constexpr uint32_t WK_BYTES = DN * 128;          // W_UK chunk [128 d x 64 c], K-major
-constexpr uint32_t WV_BYTES = 64 * DV * 2;       // W_UV chunk [64 c x 128 e], two MN-major blocks
-constexpr uint32_t STAGE_BYTES = WK_BYTES + WV_BYTES;   // 32768
-constexpr int STAGES = 3;
+// per CTA of the pair, half of each W chunk: W_UK rows d = 64 r .. 64 r + 63 (K-major
+// [64 d x 64 c]) and W_UV columns e = 64 r .. 64 r + 63 (one MN-major [64 c x 64 e] block)
+constexpr uint32_t WK_BYTES = 64 * 128;
+constexpr uint32_t WV_BYTES = 64 * 128;
+constexpr uint32_t STAGE_BYTES = WK_BYTES + WV_BYTES;   // 16384
+constexpr int STAGES = 6;
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_STAGE = A_BYTES;
 constexpr uint32_t OFF_MISC = OFF_STAGE + STAGES * STAGE_BYTES;
 constexpr uint32_t MISC_BYTES = 1024;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES;   // the base is 1 KB aligned (checked)
 constexpr uint32_t TMEM_COLS = 512;              // two buffers of [K_nope 128 | V 128]
-constexpr uint32_t IDESC_K = ptx::idesc_bf16(128, DN, 0, 0);
-constexpr uint32_t IDESC_V = ptx::idesc_bf16(128, DV, 0, 1);
-constexpr int THREADS = 192;                     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+// 2-SM MMAs: M = 256 (each CTA's 128 tokens), N = 128 split 64 / 64 between the CTAs
+constexpr uint32_t IDESC_K = ptx::idesc_bf16(256, DN, 0, 0);
+constexpr uint32_t IDESC_V = ptx::idesc_bf16(256, DV, 0, 1);
+constexpr int THREADS = 192;                     // warp 0 TMA, warp 1 MMA (leader), warps 2..5 epilogue
 static_assert(SMEM_BYTES <= 232448, "smem");
 static_assert((OFF_STAGE % 1024) == 0 && (STAGE_BYTES % 1024) == 0, "align");
 
 struct Misc {
-    uint64_t a_full;
-    uint64_t w_full[STAGES], w_empty[STAGES];
-    uint64_t d_full[2], d_free[2];
+    uint64_t a_full;                 // leader: both CTAs' c_KV tiles landed
+    uint64_t w_full[STAGES];         // leader: both halves of a W chunk landed
+    uint64_t w_empty[STAGES];        // each CTA: the chunk's MMAs are done
+    uint64_t d_full[2];              // each CTA: a head's products are in tensor memory
+    uint64_t d_free[2];              // leader: both CTAs' epilogues have read them
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -76,115 +81,134 @@ struct DecompressArgs {
     __nv_bfloat16 *k_nope;       // [B, H, Lpad, 128]
     __nv_bfloat16 *v;            // [B, H, Lpad, 128]
     int64_t timeout_ns;
-    int32_t batch, heads, max_pages, num_pages, l_pad, tiles_per_seq, heads_per_cta;
+    int32_t batch, heads, max_pages, num_pages, l_pad, pairs_per_seq, heads_per_cta;
 };
 
-// kFp8: the c_KV tile comes from the E4M3 cache; the four epilogue warps
-// dequantise it into the resident shared-memory tile before the first MMA
-// (bf16(value(code) * scale), the cache's dequantisation), so the rest of the
-// kernel is unchanged. map_ckv is unused then.
+// A CTA pair (cluster of two) covers tiles 2p and 2p + 1 of a sequence for a group
+// of heads; the leader issues 2-SM MMAs with M = 256, each CTA supplying its own
+// 128-token c_KV tile (A) and half of every W chunk (B), so each SM streams half
+// the weight bytes of a one-CTA design for the same work. kFp8: the c_KV tiles
+// come from the E4M3 cache; the epilogue warps dequantise them into the resident
+// shared-memory tile before the first MMA (bf16(value(code) * scale)), so the rest
+// is unchanged. map_ckv is unused then.
 template <bool kFp8>
-__global__ void __launch_bounds__(dkv::THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dkv::THREADS, 1)
     decompress_kernel(const __grid_constant__ CUtensorMap map_ckv,
                       const __grid_constant__ CUtensorMap map_wuk,
                       const __grid_constant__ CUtensorMap map_wuv, const DecompressArgs args) {
     using namespace dkv;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_base = ptx::smem_u32(smem_raw);
-    const uint32_t base = (raw_base + 1023u) & ~1023u;
-    uint8_t *smem = smem_raw + (base - raw_base);
-    dkv::Misc *misc = reinterpret_cast<dkv::Misc *>(smem + OFF_MISC);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = ptx::smem_u32(smem_raw);
+    if (base & 1023u) {            // swizzled operands need a 1 KB aligned base; uniform over the pair
+        if (threadIdx.x == 0) record_error(kErrUnsupported);
+        return;
+    }
+    dkv::Misc *misc = reinterpret_cast<dkv::Misc *>(smem_raw + OFF_MISC);
     volatile int32_t *abort_flag = &misc->abort_flag;
     auto bar = [&](const uint64_t *b) { return ptx::smem_u32(b); };
+    auto leader_bar = [&](const uint64_t *b) { return ptx::mapa(ptx::smem_u32(b), 0); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int32_t b = blockIdx.x / args.tiles_per_seq;
-    const int32_t tb = blockIdx.x - b * args.tiles_per_seq;
+    const uint32_t rank = ptx::cluster_ctarank();      // 0 = leader
+    const int32_t pair = blockIdx.x >> 1;
+    const int32_t b = pair / args.pairs_per_seq;
+    const int32_t tb = 2 * (pair - b * args.pairs_per_seq) + static_cast<int32_t>(rank);
     const int32_t h0 = blockIdx.y * args.heads_per_cta;
     const int32_t nh = min(args.heads_per_cta, args.heads - h0);
-    int32_t L = args.seq_lens[b];
+    const int32_t L = args.seq_lens[b];
+    // early exits are uniform over the pair (same sequence, same head group)
     if (L < 0 || static_cast<int64_t>(L) > static_cast<int64_t>(args.max_pages) * 64) {
-        if (threadIdx.x == 0 && tb == 0 && blockIdx.y == 0) record_error(kErrDeviceBounds);
+        if (threadIdx.x == 0 && rank == 0 && tb == 0 && blockIdx.y == 0) record_error(kErrDeviceBounds);
         return;
     }
-    if (TOK * tb >= L || nh <= 0) return;          // tile past the sequence: never read
+    if (TOK * (tb - static_cast<int32_t>(rank)) >= L || nh <= 0) return;   // the pair's first tile
+    const int32_t rows_written = (L + TOK - 1) / TOK * TOK;   // rows >= L of the last tile are zeros
+    const int32_t npages = (L + 63) / 64;
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(bar(&misc->a_full), kFp8 ? 4 : 1);
+        ptx::mbar_init(bar(&misc->a_full), kFp8 ? 8 : 1);
         for (int i = 0; i < STAGES; ++i) {
             ptx::mbar_init(bar(&misc->w_full[i]), 1);
             ptx::mbar_init(bar(&misc->w_empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(&misc->d_full[i]), 1);
-            ptx::mbar_init(bar(&misc->d_free[i]), 4);
+            ptx::mbar_init(bar(&misc->d_free[i]), 8);
         }
         ptx::mbar_init(bar(&misc->drain), 1);
         misc->abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc<1>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
-        ptx::tmem_relinquish<1>();
+        ptx::tmem_alloc<2>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
+        ptx::tmem_relinquish<2>();
     }
     ptx::tc_fence_before();
     __syncthreads();
+    ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const int total = nh * CHUNKS;                 // W chunks streamed by this CTA
+    const int total = nh * CHUNKS;                 // W chunks streamed by the pair
+    const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
+    // pages of this CTA's tile; a tile past the sequence (the pair's second) re-reads the
+    // sequence's first page: its products are computed but never stored
+    auto tile_page = [&](int i, bool *bad) -> int32_t {
+        int32_t pi = 2 * tb + i;                   // page index within the sequence
+        if (pi >= npages) pi = (2 * tb < npages) ? 2 * tb : 0;   // npages >= 1 here
+        int32_t pg = trow[pi];
+        if (pg < 0 || pg >= args.num_pages) { *bad = true; pg = 0; }
+        return pg;
+    };
 
     if (warp == 0) {
         if (ptx::elect_one()) {
             if (!kFp8) ptx::prefetch_tensormap(&map_ckv);
             ptx::prefetch_tensormap(&map_wuk);
             ptx::prefetch_tensormap(&map_wuv);
-            const uint32_t ab = bar(&misc->a_full);
+            const uint32_t ab = rank == 0 ? bar(&misc->a_full) : leader_bar(&misc->a_full);
             if (!kFp8) {
-                const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
-                const int32_t npages = (L + 63) / 64;
-                int32_t pg[2] = {trow[2 * tb], (2 * tb + 1 < npages) ? trow[2 * tb + 1] : -1};
                 bool bad = false;
-                if (pg[0] < 0 || pg[0] >= args.num_pages) { bad = true; pg[0] = 0; }
-                if (pg[1] == -1 && !(2 * tb + 1 < npages)) pg[1] = pg[0];   // rows >= L: zeroed on store
-                else if (pg[1] < 0 || pg[1] >= args.num_pages) { bad = true; pg[1] = 0; }
+                const int32_t pg[2] = {tile_page(0, &bad), tile_page(1, &bad)};
                 if (bad) record_error(kErrDeviceBounds);
-                ptx::mbar_arrive_expect_tx(ab, A_BYTES);
+                if (rank == 0) ptx::mbar_arrive_expect_tx(ab, 2 * A_BYTES);
                 for (int blk = 0; blk < CHUNKS; ++blk)
                     for (int i = 0; i < 2; ++i)
-                        ptx::tma_load_3d(base + OFF_A + blk * (TOK * 128) + i * (64 * 128), &map_ckv,
-                                         ab, 64 * blk, 0, pg[i]);
+                        ptx::tma_load_3d_pair(base + OFF_A + blk * (TOK * 128) + i * (64 * 128),
+                                              &map_ckv, ab, 64 * blk, 0, pg[i]);
             }
             int n = 0;
             for (; n < total; ++n) {
                 const int st = n % STAGES;
-                if (n >= STAGES && !wait_bounded<false>(bar(&misc->w_empty[st]),
-                                                        ((n / STAGES) - 1) & 1, abort_flag,
-                                                        args.timeout_ns))
+                if (n >= STAGES && !wait_bounded<true>(bar(&misc->w_empty[st]),
+                                                       ((n / STAGES) - 1) & 1, abort_flag,
+                                                       args.timeout_ns))
                     break;
                 const int32_t h = h0 + n / CHUNKS;
                 const int c = n % CHUNKS;
-                const uint32_t fb = bar(&misc->w_full[st]);
+                const uint32_t fb = rank == 0 ? bar(&misc->w_full[st]) : leader_bar(&misc->w_full[st]);
                 const uint32_t sb = base + OFF_STAGE + st * STAGE_BYTES;
-                ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                ptx::tma_load_3d(sb, &map_wuk, fb, 64 * c, 0, h);
-                ptx::tma_load_3d(sb + WK_BYTES, &map_wuv, fb, 0, 64 * c, h);
-                ptx::tma_load_3d(sb + WK_BYTES + 64 * 128, &map_wuv, fb, 64, 64 * c, h);
+                if (rank == 0) ptx::mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+                ptx::tma_load_3d_pair(sb, &map_wuk, fb, 64 * c, 64 * rank, h);
+                ptx::tma_load_3d_pair(sb + WK_BYTES, &map_wuv, fb, 64 * rank, 64 * c, h);
             }
-            // no copy may still be landing when the CTA exits (the abort path)
-            if (!kFp8) wait_bounded<false>(ab, 0, abort_flag, args.timeout_ns);
-            for (int m = (n > STAGES ? n - STAGES : 0); m < n; ++m)
-                wait_bounded<false>(bar(&misc->w_full[m % STAGES]), (m / STAGES) & 1, abort_flag,
-                                    args.timeout_ns);
+            // no copy may still be landing when the CTA exits (the abort path): the leader
+            // waits for the pair's last copies
+            if (rank == 0) {
+                if (!kFp8) wait_bounded<true>(ab, 0, abort_flag, args.timeout_ns);
+                for (int m = (n > STAGES ? n - STAGES : 0); m < n; ++m)
+                    wait_bounded<true>(bar(&misc->w_full[m % STAGES]), (m / STAGES) & 1, abort_flag,
+                                       args.timeout_ns);
+            }
         }
     } else if (warp == 1) {
-        if (ptx::elect_one()) {
-            bool ok = wait_bounded<false>(bar(&misc->a_full), 0, abort_flag, args.timeout_ns);
+        if (rank == 0 && ptx::elect_one()) {
+            bool ok = wait_bounded<true>(bar(&misc->a_full), 0, abort_flag, args.timeout_ns);
             int n = 0;
             for (int j = 0; ok && j < nh; ++j) {
                 const int u = j & 1;
-                if (j >= 2 && !wait_bounded<false>(bar(&misc->d_free[u]), ((j >> 1) - 1) & 1,
-                                                   abort_flag, args.timeout_ns)) {
+                if (j >= 2 && !wait_bounded<true>(bar(&misc->d_free[u]), ((j >> 1) - 1) & 1,
+                                                  abort_flag, args.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -192,8 +216,8 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
                 const uint32_t dk = tmem + 256u * u, dv = dk + 128u;
                 for (int c = 0; c < CHUNKS; ++c, ++n) {
                     const int st = n % STAGES;
-                    if (!wait_bounded<false>(bar(&misc->w_full[st]), (n / STAGES) & 1, abort_flag,
-                                             args.timeout_ns)) {
+                    if (!wait_bounded<true>(bar(&misc->w_full[st]), (n / STAGES) & 1, abort_flag,
+                                            args.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -205,24 +229,24 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
                         const uint64_t a = ptx::smem_desc(base + OFF_A + c * (TOK * 128) + kk * 32,
                                                           16, 1024, ptx::kSwizzle128B);
                         const uint64_t bk = ptx::smem_desc(sb + kk * 32, 16, 1024, ptx::kSwizzle128B);
-                        ptx::mma_bf16_ss<1>(dk, a, bk, IDESC_K, acc);
+                        ptx::mma_bf16_ss<2>(dk, a, bk, IDESC_K, acc);
                         const uint64_t bv = ptx::smem_desc(sb + WK_BYTES + kk * 2048, 64 * 128, 1024,
                                                            ptx::kSwizzle128B);
-                        ptx::mma_bf16_ss<1>(dv, a, bv, IDESC_V, acc);
+                        ptx::mma_bf16_ss<2>(dv, a, bv, IDESC_V, acc);
                     }
-                    ptx::mma_commit(bar(&misc->w_empty[st]));
+                    ptx::mma_commit_pair(bar(&misc->w_empty[st]), 0x3);
                 }
                 if (!ok) break;
-                ptx::mma_commit(bar(&misc->d_full[u]));
+                ptx::mma_commit_pair(bar(&misc->d_full[u]), 0x3);
             }
-            ptx::mma_commit(bar(&misc->drain));
-            wait_bounded<false>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
+            ptx::mma_commit_pair(bar(&misc->drain), 0x1);
+            wait_bounded<true>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
         }
     } else {
+        const uint32_t remote_arrive_a = rank == 0 ? bar(&misc->a_full) : leader_bar(&misc->a_full);
         if (kFp8) {
             // dequantise this warp's 32 tile rows: one 512-byte row per warp load
             // (16 codes per lane), written as two swizzled 16-byte chunks per lane
-            const int32_t *trow = args.block_table + static_cast<int64_t>(b) * args.max_pages;
             bool bad = false;
             for (int rr = 0; rr < 32; ++rr) {
                 const int r = 32 * (warp - 2) + rr;
@@ -248,17 +272,23 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
             if (bad && lane == 0) record_error(kErrDeviceBounds);
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(&misc->a_full));
+            if (lane == 0) {
+                if (rank == 0) ptx::mbar_arrive(remote_arrive_a);
+                else ptx::mbar_arrive_cluster(remote_arrive_a);
+            }
         }
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int32_t t = TOK * tb + row;
         const bool live = t < L;
+        const bool store = t < rows_written;
         const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const uint32_t dfree = [&] {
+            return rank == 0 ? ptx::smem_u32(&misc->d_free[0]) : ptx::mapa(ptx::smem_u32(&misc->d_free[0]), 0);
+        }();
         for (int j = 0; j < nh; ++j) {
             const int u = j & 1;
-            if (!wait_bounded<false>(bar(&misc->d_full[u]), (j >> 1) & 1, abort_flag,
-                                     args.timeout_ns))
+            if (!wait_bounded<true>(bar(&misc->d_full[u]), (j >> 1) & 1, abort_flag, args.timeout_ns))
                 break;
             ptx::tc_fence_after();
             const int64_t rowoff =
@@ -266,14 +296,16 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
 #pragma unroll 1
             for (int part = 0; part < 2; ++part) {
                 __nv_bfloat16 *dst = (part ? args.v : args.k_nope) + rowoff;
-#pragma unroll 1
-                for (int cch = 0; cch < 4; ++cch) {
-                    uint32_t r[32];
-                    ptx::tmem_ld32(tmem + lane_base + 256u * u + 128u * part + 32u * cch, r);
-                    ptx::tmem_wait_ld();
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cch);
+                uint32_t r[128];                    // this part's 128 columns, one wait
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                for (int cch = 0; cch < 4; ++cch)
+                    ptx::tmem_ld32(tmem + lane_base + 256u * u + 128u * part + 32u * cch,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&r[32 * cch]));
+                ptx::tmem_wait_ld();
+                if (store) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
                         uint4 w = make_uint4(0, 0, 0, 0);
                         if (live)
                             w = make_uint4(
@@ -287,13 +319,18 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(&misc->d_free[u]));
+            if (lane == 0) {
+                const uint32_t fb = dfree + 8u * u;
+                if (rank == 0) ptx::mbar_arrive(fb);
+                else ptx::mbar_arrive_cluster(fb);
+            }
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    ptx::cluster_sync();
     ptx::tc_fence_after();
-    if (warp == 1) ptx::tmem_dealloc<1>(tmem, TMEM_COLS);
+    if (warp == 1) ptx::tmem_dealloc<2>(tmem, TMEM_COLS);
 }
 
 // ===========================================================================
