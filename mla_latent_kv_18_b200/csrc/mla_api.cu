@@ -728,11 +728,16 @@ mla_status mla_decompress_kv_fp8(const mla_dims *dims, const mla_pool *ckv8, con
                              workspace_bytes, stream);
 }
 
-mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
-                                 const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
-                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
-                                 const void *workspace, size_t workspace_bytes, void *out,
-                                 float *lse, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Every argument check of mla_prefill_attention (host only, nothing launched).
+mla_status check_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
+                                   const mla_pool *kr, int32_t num_pages,
+                                   const int32_t *block_table, int32_t max_pages_per_seq,
+                                   const int32_t *seq_lens, int32_t batch, const void *workspace,
+                                   size_t workspace_bytes, const void *out, const float *lse) {
     mla_status st = check_prefill_dims(dims);
     if (st != MLA_OK) return st;
     if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
@@ -750,6 +755,24 @@ mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const vo
     if (batch > 65535 || H > 65535 || q_blocks > (int64_t(1) << 31) - 1 ||
         static_cast<int64_t>(batch) * M > (int64_t(1) << 31) - 1)
         return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_prefill_attention(const mla_dims *dims, const void *q_c, const void *q_r,
+                                 const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                                 int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                                 const void *workspace, size_t workspace_bytes, void *out,
+                                 float *lse, void *stream) {
+    mla_status st = check_prefill_attention(dims, q_c, q_r, kr, num_pages, block_table,
+                                            max_pages_per_seq, seq_lens, batch, workspace,
+                                            workspace_bytes, out, lse);
+    if (st != MLA_OK || batch == 0) return st;
+    const int64_t M = dims->n_q, H = dims->num_heads;
+    const int64_t q_blocks = (M + mla::pfa::ROWS - 1) / mla::pfa::ROWS;
     if ((st = device_ready()) != MLA_OK) return st;
     const int64_t l_pad = prefill_l_pad(max_pages_per_seq);
     const uint64_t BM = static_cast<uint64_t>(batch) * M, BH = static_cast<uint64_t>(batch) * H;
@@ -793,12 +816,11 @@ mla_status mla_prefill(const mla_dims *dims, const void *q_c, const void *q_r, c
                        int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
                        const void *w_uk, const void *w_uv, void *workspace,
                        size_t workspace_bytes, void *out, float *lse, void *stream) {
-    mla_status st = check_prefill_dims(dims);
-    if (st != MLA_OK) return st;
-    if (batch < 0 || max_pages_per_seq <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
-    if (batch == 0) return MLA_OK;
-    if (!q_c || !q_r || !out) return MLA_ERR_INVALID_ARG;
-    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    // both steps' arguments are checked before the first launch
+    mla_status st = check_prefill_attention(dims, q_c, q_r, kr, num_pages, block_table,
+                                            max_pages_per_seq, seq_lens, batch, workspace,
+                                            workspace_bytes, out, lse);
+    if (st != MLA_OK || batch == 0) return st;
     if ((st = mla_decompress_kv(dims, ckv, num_pages, block_table, max_pages_per_seq, seq_lens,
                                 batch, w_uk, w_uv, workspace, workspace_bytes, stream)) != MLA_OK)
         return st;

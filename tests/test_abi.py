@@ -182,6 +182,12 @@ def test_prefill_workspace_size_and_validation_without_launch(b):
                                  ctypes.c_void_p(0x1010), ws, null) == 1   # not 256-B aligned
     assert lib.mla_prefill_attention(by(d), ctypes.c_void_p(0x1002), fake, by(kpool), 4, fake, 2,
                                      fake, 2, fake, ws, fake, null, null) == 1   # misaligned q_c
+    # mla_prefill checks the attention step's arguments before launching the decompression:
+    # everything valid except a misaligned output is refused without touching a device
+    wsp = ctypes.c_void_p(0x100000)
+    ok_args = [fake, fake, by(pool), by(kpool), 4, fake, 2, fake, 2, fake, fake, wsp, ws]
+    assert lib.mla_prefill(by(d), *ok_args, ctypes.c_void_p(0x1008), null, null) == 1
+    assert lib.mla_prefill(by(d), *ok_args, fake, ctypes.c_void_p(0x1002), null) == 1
 
 
 def test_cache_write_and_fp8_calls_validate_without_launch(b):
