@@ -472,6 +472,9 @@ mla_status mla_decode_latent_noalloc(const mla_dims *dims, const void *q, const 
     if (batch == 0) return MLA_OK;
     const size_t need = mla_decode_workspace_bytes(dims, batch, num_parts);
     if (need == 0 || need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_INVALID_ARG;
+    // the combine's own output checks, before the decode is launched
+    if (!o_lat || !aligned(o_lat, 16) || (lse_out && !aligned(lse_out, 4)))
+        return MLA_ERR_INVALID_ARG;
     if ((st = device_ready()) != MLA_OK) return st;
     void *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != MLA_OK) return st;

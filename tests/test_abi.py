@@ -230,3 +230,18 @@ def test_cache_write_and_fp8_calls_validate_without_launch(b):
     short = b.MLAPool(0x1000, 64 * 256, 256)
     assert lib.mla_decompress_kv_fp8(by(dp), by(short), fake, 4, fake, 2, fake, 2, fake, fake,
                                      fake, ws, null) == 1
+
+
+def test_noalloc_decode_checks_outputs_before_launching(b):
+    # a misaligned or missing o_lat (or lse_out) is refused before the split-KV decode is
+    # launched, so nothing touches a device
+    lib = b.lib
+    by = ctypes.byref
+    d = _dims(b)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x1000)
+    pool = b.MLAPool(0x1000, 64 * 576, 576)
+    args = [fake, by(pool), by(pool), 4, fake, 2, fake, 2, 4]
+    assert lib.mla_decode_latent_noalloc(by(d), *args, null, null, null) == 1
+    assert lib.mla_decode_latent_noalloc(by(d), *args, ctypes.c_void_p(0x1004), null, null) == 1
+    assert lib.mla_decode_latent_noalloc(by(d), *args, fake, ctypes.c_void_p(0x1002), null) == 1
