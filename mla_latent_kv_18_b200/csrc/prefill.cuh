@@ -7,12 +7,13 @@
 // fewer FLOPs than the latent width (576 and 512). Two kernels:
 //
 //  * decompress_kernel: K_nope[b,h,t,:] = c_KV[t] W_UK[h]^T and
-//    V[b,h,t,:] = c_KV[t] W_UV[h] ("MHA2MLA" page §2.1) for 128-token tiles.
-//    One CTA keeps its tile of c_KV (128 tokens x 512 channels, two pages) in
-//    shared memory, streams W_UK[h] / W_UV[h] in 64-channel chunks through a
-//    TMA ring for each head of its group, and accumulates both products with
-//    tcgen05 MMAs into a double-buffered tensor-memory tile, so that the
-//    epilogue of one head overlaps the MMAs of the next.
+//    V[b,h,t,:] = c_KV[t] W_UV[h] ("MHA2MLA" page §2.1). A CTA pair covers two
+//    128-token tiles: each CTA keeps its tile of c_KV (128 tokens x 512
+//    channels, two pages) in shared memory and streams its half of W_UK[h] /
+//    W_UV[h] in 64-channel chunks through a TMA ring for each head of its
+//    group; the leader accumulates both products with 2-SM tcgen05 MMAs
+//    (M = 256) into double-buffered tensor-memory tiles, so that the epilogue
+//    of one head overlaps the MMAs of the next.
 //  * prefill_attn_kernel: causal attention of 128 queries of one (sequence,
 //    head) against the decompressed keys [K_nope | k_R] and values V: scores
 //    in tensor memory (two buffers), fp32 online softmax in the exp2 domain by
