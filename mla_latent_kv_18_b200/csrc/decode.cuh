@@ -164,6 +164,7 @@ struct Misc {
     uint64_t drain;                   // MMA drain before tensor memory is freed
     uint64_t qk_full[pair::QK_STAGES], qk_empty[pair::QK_STAGES];   // the pair kernel's two rings
     uint64_t pv_full[pair::PV_STAGES], pv_empty[pair::PV_STAGES];
+    uint64_t pv_landed[pair::PV_STAGES];   // pair kernel: a P.V slot has landed (both CTAs)
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t cur_b;
@@ -208,6 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int i = 0; i < PV_STAGES; ++i) {
             ptx::mbar_init(bar(&misc->pv_full[i]), 1);
             ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
+            ptx::mbar_init(bar(&misc->pv_landed[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(&misc->s_full[i]), 1);
@@ -327,6 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             int64_t tq = q_has ? wq.t_begin : 0, tp = p_has ? wp.t_begin : 0;
             int64_t kq = 0, kp = 0, gq = 0, gp = 0;
             bool q_ready_seen = false, o_free_seen = false;
+            bool landed_sent = false;   // landing of P.V slot kp forwarded to both CTAs
             uint64_t idle_since = ptx::globaltimer_ns();
             uint32_t spins = 0;
             while ((q_has || p_has) && !*abort_flag) {
@@ -376,9 +379,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         o_free_seen = ptx::mbar_test_wait(bar(&misc->o_free), (gp - 1) & 1);
                     const int s = static_cast<int>(kp & 1);            // P buffer, score buffer
                     const int ps = static_cast<int>(kp % PV_STAGES);   // P.V operand slot
-                    if ((!first || gp == 0 || o_free_seen) &&
-                        ptx::mbar_test_wait(bar(&misc->pv_full[ps]), (kp / PV_STAGES) & 1) &&
+                    // Once both CTAs' copies of slot ps have landed, say so to each
+                    // CTA: the softmax warps clear the rows past a sequence's end in
+                    // its last tile before they report P ready.
+                    if (!landed_sent &&
+                        ptx::mbar_test_wait(bar(&misc->pv_full[ps]), (kp / PV_STAGES) & 1)) {
+                        ptx::mbar_arrive(bar(&misc->pv_landed[ps]));
+                        ptx::mbar_arrive_cluster(ptx::mapa(bar(&misc->pv_landed[ps]), 1));
+                        landed_sent = true;
+                        progressed = true;
+                    }
+                    if (landed_sent && (!first || gp == 0 || o_free_seen) &&
                         ptx::mbar_test_wait(bar(&misc->p_ready[s]), (kp >> 1) & 1)) {
+                        landed_sent = false;
                         ptx::tc_fence_after();
                         const uint64_t a0 = ptx::smem_desc(base + OFF_P + s * P_BYTES, 16, 1024,
                                                            ptx::kSwizzle128B);
@@ -570,6 +583,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                  pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
                                  pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
                                  pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+                }
+                // Last tile of the sequence: the page's rows past its end were loaded
+                // with the page and may hold any bits (an unwritten or recycled page
+                // slot). Their P is 0, but 0 * NaN = NaN in the value product, so
+                // they are cleared in this CTA's P.V slot once it has landed.
+                const int32_t valid = L - static_cast<int32_t>(t) * TOK;
+                if (valid < TOK) {
+                    const int ps = static_cast<int>(k % PV_STAGES);
+                    if (!wait_bounded(bar(&misc->pv_landed[ps]), (k / PV_STAGES) & 1, abort_flag,
+                                      args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t slot_base = base + OFF_PV + ps * STAGE_PV;
+                    const int n16 = (TOK - valid) * 8;   // 16-byte chunks per channel block
+                    for (int idx = st_tid; idx < 4 * n16; idx += 128) {
+                        const int u = idx / n16, rem = idx - u * n16;
+                        st_shared_v4(slot_base + u * (TOK * 128) + (valid + (rem >> 3)) * 128 +
+                                         (rem & 7) * 16,
+                                     0u, 0u, 0u, 0u);
+                    }
                 }
                 ptx::fence_proxy_async_smem();
                 if (any_need) ptx::tc_fence_before();   // order the O rescale stores
@@ -969,8 +1003,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                      pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
                                      pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
                     }
-                    ptx::fence_proxy_async_smem();
                 }
+                // Last tile of the sequence: the stage's c_KV rows past its end (the
+                // tail of the last page, or a second page not loaded for this tile)
+                // may hold any bits; P is 0 there, but 0 * NaN = NaN in the value
+                // product, so they are cleared. QK^T of this tile has finished
+                // reading the stage (s_full) and P.V waits for p_ready.
+                const int32_t valid = L - static_cast<int32_t>(t) * TOK;
+                if (valid < TOK) {
+                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    for (int idx = st_tid; idx < (TOK - valid) * 8; idx += 128)
+                        st_shared_v4(st + (valid + (idx >> 3)) * 128 + (idx & 7) * 16, 0u, 0u, 0u, 0u);
+                }
+                ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
                 arrive(&misc->p_ready[s]);
             }
