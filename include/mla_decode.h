@@ -108,6 +108,22 @@ int32_t mla_decode_num_parts(const mla_dims *dims, int64_t total_tiles, int32_t 
  * Returns 0 for invalid dims. */
 size_t mla_decode_workspace_bytes(const mla_dims *dims, int32_t batch, int32_t num_parts);
 
+/* The same two sizing helpers in split-KV terms (a split is one partition),
+ * sized from the batch and its longest sequence instead of the tile total:
+ *   mla_default_num_splits(dims, batch, max_seq_len, num_sms)
+ *       = mla_decode_num_parts(dims, batch * ceil(max_seq_len / tile), num_sms)
+ *     with tile = 64 tokens (d_latent 512) or 128 (d_latent 64), i.e. the
+ *     partition count for `batch` sequences of at most max_seq_len tokens;
+ *     returns >= 1 (1 for invalid arguments).
+ *   mla_decode_workspace_size(dims, batch, num_splits)
+ *       = mla_decode_workspace_bytes(dims, batch, num_splits).
+ * The partials of every split live inside the workspace at the layout given
+ * above, so mla_decode_splitkv and mla_combine take the workspace instead of
+ * separate partial-output pointers. */
+int32_t mla_default_num_splits(const mla_dims *dims, int32_t batch, int32_t max_seq_len,
+                               int32_t num_sms);
+size_t mla_decode_workspace_size(const mla_dims *dims, int32_t batch, int32_t num_splits);
+
 /*
  * Split-KV decode in latent space (the absorbed score and value steps).
  * The flattened list of tiles of all sequences (N tiles of 64 tokens for

@@ -20,7 +20,8 @@ EXPORTS = ("mla_absorb_q", "mla_decode_num_parts", "mla_decode_workspace_bytes",
            "mla_decode_latent_noalloc", "mla_debug_gather", "mla_combine_absorb_out",
            "mla_absorb_q_rope", "mla_prefill_workspace_bytes", "mla_decompress_kv",
            "mla_prefill_attention", "mla_prefill", "mla_append_kv",
-           "mla_append_kv_fp8", "mla_gather_dequant_fp8", "mla_decompress_kv_fp8")
+           "mla_append_kv_fp8", "mla_gather_dequant_fp8", "mla_decompress_kv_fp8",
+           "mla_default_num_splits", "mla_decode_workspace_size")
 
 
 class MLADims(ctypes.Structure):
@@ -72,6 +73,8 @@ def _load():
                                     P]),
         "mla_gather_dequant_fp8": (i32, [PL, P, i32, i32, P, i32, P, i32, i32, P, P]),
         "mla_decompress_kv_fp8": (i32, [D, PL, P, i32, P, i32, P, i32, P, P, P, sz, P]),
+        "mla_default_num_splits": (i32, [D, i32, i32, i32]),
+        "mla_decode_workspace_size": (sz, [D, i32, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

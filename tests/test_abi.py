@@ -106,6 +106,19 @@ def test_num_parts_and_workspace(b):
     assert ws == o + (slots * R * 4 + 255) // 256 * 256
     bad = _dims(b, d_latent=256)
     assert lib.mla_decode_workspace_bytes(ctypes.byref(bad), 16, 74) == 0
+    # the split-KV-named helpers are the same arithmetic
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 16, 74) == ws
+    assert lib.mla_default_num_splits(ctypes.byref(d), 16, 65536, 148) == 74
+    assert lib.mla_default_num_splits(ctypes.byref(d), 1, 256, 148) == 1
+    for batch, L in ((3, 1000), (64, 32768), (2, 1)):
+        tiles = batch * ((L + 63) // 64)
+        assert lib.mla_default_num_splits(ctypes.byref(d), batch, L, 148) == \
+            lib.mla_decode_num_parts(ctypes.byref(d), tiles, 148)
+    r = _dims(b, n_q=2, num_heads=32, d_nope=120, d_latent=64, d_rope=8)
+    assert lib.mla_default_num_splits(ctypes.byref(r), 32, 8192, 148) > 1
+    assert lib.mla_default_num_splits(ctypes.byref(r), 32, 8192, 148) == \
+        lib.mla_decode_num_parts(ctypes.byref(r), 32 * 64, 148)
+    assert lib.mla_default_num_splits(ctypes.byref(bad), 16, 4096, 148) == 1
 
 
 def test_argument_validation_without_launch(b):
