@@ -39,6 +39,8 @@ UNIT = "KV-tokens/s"
 PREFILL_METRIC = "MLA prefill (decompress branch) query tokens/s per B200 (bf16) + % of tensor roofline"
 PREFILL_UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+# working set per step kept above three times the 126 MB L2
+L2_FLUSH_BYTES = 3 * 126 * 1024 * 1024
 FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM bytes per launch of the decode kernel from an ncu capture, keyed by the
@@ -358,24 +360,34 @@ def main():
     dec = api.Decoder(dims, w.batch, d["block_table"].shape[1], total_tiles, dev)
     stream = torch.cuda.current_stream()
     tokens_per_step = float(lens.sum())
+    # Model state of one layer: the latent cache and the two absorbed weights. When
+    # it fits in L2, the steps walk over several layers' copies (a model's layers
+    # each own a cache and weights), so that no step finds its operands in L2.
+    state_keys = ("ckv_pool", "kr_pool", "w_uk", "w_uv")
+    layer_bytes = sum(d[k].numel() * d[k].element_size() for k in state_keys)
+    n_layers = max(1, math.ceil(L2_FLUSH_BYTES / layer_bytes))
+    layers = [d] + [{k: d[k].clone() for k in state_keys} for _ in range(n_layers - 1)]
+    cursor = [0]
 
     def step(ev=None, x=None, out=None):
         x = d if x is None else x            # this step's inputs (q_c, q_r, table, lengths)
         out = dec.out if out is None else out
-        api.absorb_q(x["q_c"], x["q_r"], d["w_uk"], dims, out=dec.q)
+        m = layers[cursor[0] % n_layers]     # this step's layer (cache and weights)
+        cursor[0] += 1
+        api.absorb_q(x["q_c"], x["q_r"], m["w_uk"], dims, out=dec.q)
         if ev is not None:
             ev[0].record(stream)
-        api.decode_splitkv(dec.q, d["ckv_pool"], d["kr_pool"], x["block_table"], x["seq_lens"],
+        api.decode_splitkv(dec.q, m["ckv_pool"], m["kr_pool"], x["block_table"], x["seq_lens"],
                            dims, dec.num_parts, workspace=dec.workspace)
         if ev is not None:
             ev[1].record(stream)
         if a.unfused:
             api.combine(dec.workspace, x["seq_lens"], dec.max_pages, dims, dec.num_parts,
                         o_lat=dec.o_lat, lse_out=dec.lse)
-            api.absorb_out(dec.o_lat, d["w_uv"], dims, out=out)
+            api.absorb_out(dec.o_lat, m["w_uv"], dims, out=out)
         else:
             api.combine_absorb_out(dec.workspace, x["seq_lens"], dec.max_pages, dims,
-                                   dec.num_parts, d["w_uv"], out=out, lse_out=dec.lse)
+                                   dec.num_parts, m["w_uv"], out=out, lse_out=dec.lse)
 
     def barrier():
         if world > 1:
@@ -501,7 +513,12 @@ def main():
             "config": {"workload": _workload_desc(w, lens), "batch": w.batch,
                        "seq_len": w.seq_len or list(w.ragged), "heads": w.heads,
                        "kv_tokens_per_step": tokens_per_step, "num_parts": dec.num_parts,
-                       "l2": "inputs larger than L2 (latent cache %.2f GB), no flush" % (kv_bytes / 1e9),
+                       "l2": ("inputs larger than L2 (latent cache %.2f GB), no flush" % (kv_bytes / 1e9)
+                              if n_layers == 1 else
+                              "inputs larger than L2: steps cycle over %d layers' copies of the "
+                              "latent cache and weights (%.2f GB in all), no flush"
+                              % (n_layers, n_layers * layer_bytes / 1e9)),
+                       "layers": n_layers,
                        "parallelism": "replicas" if world > 1 else "single",
                        "step_calls": ["mla_absorb_q", "mla_decode_splitkv"] +
                                      (["mla_combine", "mla_absorb_out"] if a.unfused
