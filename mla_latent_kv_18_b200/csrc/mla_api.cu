@@ -5,7 +5,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <cstdlib>
 #include <algorithm>
 #include <mutex>
 
@@ -15,7 +14,6 @@
 #include "mla_decode.h"
 #include "common.cuh"
 #include "decode.cuh"
-#include "decode_cs.cuh"
 #include "small_kernels.cuh"
 #include "prefill.cuh"
 
@@ -81,8 +79,6 @@ mla_status device_ready() {
         if (prop.major != 10 || prop.minor != 0) { st.status = MLA_ERR_UNSUPPORTED; return; }
         if (cudaFuncSetAttribute(mla::decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::pair::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::decode_cs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 mla::cs::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_single_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::single::SMEM_BYTES) != cudaSuccess ||
@@ -144,16 +140,6 @@ mla_status pool_map(CUtensorMap *m, const mla_pool *pool, int32_t channels, int3
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
-}
-
-// Development switch for same-box A/B timing: MLA_DECODE_CS=1 runs the
-// channel-split pair kernel instead of the token-split one.
-bool legacy_pair() {
-    static const bool v = [] {
-        const char *e = std::getenv("MLA_DECODE_CS");
-        return !(e && e[0] == '1');
-    }();
-    return v;
 }
 
 mla_status launch_status() {
@@ -381,16 +367,7 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
     a.scale_log2 = a.scale * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    if (variant_of(dims) == Variant::Pair512 && !legacy_pair()) {
-        CUtensorMap mc, mkr;
-        if ((st = pool_map(&mc, ckv, 512, num_pages, 64, mla::cs::TOK,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-            return st;
-        if ((st = pool_map(&mkr, kr, 64, num_pages, mla::cs::HR, mla::cs::TOK,
-                           CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
-            return st;
-        mla::decode_cs_kernel<<<2 * num_parts, mla::cs::THREADS, mla::cs::SMEM_BYTES, s>>>(mc, mkr, a);
-    } else if (variant_of(dims) == Variant::Pair512) {
+    if (variant_of(dims) == Variant::Pair512) {
         CUtensorMap m32, m64, mkr;
         if ((st = pool_map(&m32, ckv, 512, num_pages, 64, mla::pair::OWN,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
