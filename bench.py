@@ -39,6 +39,8 @@ UNIT = "KV-tokens/s"
 PREFILL_METRIC = "MLA prefill (decompress branch) query tokens/s per B200 (bf16) + % of tensor roofline"
 PREFILL_UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+# the decode launch of every EV_EVERY-th timed step is bracketed by CUDA events
+EV_EVERY = 8
 # working set per step kept above three times the 126 MB L2
 L2_FLUSH_BYTES = 3 * 126 * 1024 * 1024
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -399,21 +401,24 @@ def main():
     torch.cuda.synchronize()
     assert api.get_device_error() == 0
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(a.steps)]
+    # the decode launch is bracketed by events on every EV_EVERY-th step only: an
+    # event between two kernels stops the next one from being launched early
+    # (programmatic dependent launch), which the other steps keep
+    evs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for i in range(0, a.steps, EV_EVERY)}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
     start.record(stream)
     for i in range(a.steps):
-        step(evs[i])
+        step(evs.get(i))
     end.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
     barrier()
     ms = start.elapsed_time(end)
-    decode_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    decode_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs.values())
     assert api.get_device_error() == 0
 
     # end to end through the same calls: every step's inputs come from pinned

@@ -55,7 +55,8 @@ struct DecodeArgs {
 };
 
 constexpr int kDecodeThreads = 192;          // single kernel: 6 warps
-constexpr int kPairThreads = 224;            // pair kernel: 7 warps (warp 6 = P.V-stage producer)
+constexpr int kPairThreads = 352;            // pair kernel: 11 warps (6 = P.V-slot producer, 7..10 segment warps)
+constexpr int kSegWarp0 = 7;                 // pair kernel: first of the four segment warps
 constexpr int kSoftmaxWarp0 = 2;             // warps 2..5
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when max grows > 2^8
 
@@ -172,6 +173,9 @@ struct Misc {
     int64_t cur_O, cur_S, cur_N;
     uint32_t xtag[2][128];            // pair kernel: tagged half-row maxima, by tile parity
     uint32_t xltag[128];              // pair kernel: tagged half-row sums, per segment
+    uint64_t q_free;                  // pair kernel: the last QK^T of a segment is done (Q may be replaced)
+    uint64_t seg_done;                // pair kernel: a segment's row sums and maxima are published
+    float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
 };
 static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
 
@@ -216,14 +220,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::mbar_init(bar(&misc->p_ready[i]), 8);
             ptx::mbar_init(bar(&misc->pv_done[i]), 1);
         }
-        ptx::mbar_init(bar(&misc->q_ready), 8);
-        ptx::mbar_init(bar(&misc->o_free), 8);
+        ptx::mbar_init(bar(&misc->q_ready), 8);     // 4 segment warps x 2 CTAs
+        ptx::mbar_init(bar(&misc->o_free), 8);      // 4 segment warps x 2 CTAs
         ptx::mbar_init(bar(&misc->drain), 1);
+        ptx::mbar_init(bar(&misc->q_free), 1);      // multicast commit from the leader
+        ptx::mbar_init(bar(&misc->seg_done), 4);    // 4 softmax warps
         misc->abort_flag = 0;
         ptx::fence_mbar_init();
     }
     for (int i = threadIdx.x; i < 3 * 128; i += blockDim.x)
         (i < 256 ? misc->xtag[i >> 7][i & 127] : misc->xltag[i - 256]) = 0u;
+    if (warp == 1) {
+        ptx::tmem_alloc<2>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
+        ptx::tmem_relinquish<2>();
+    }
+    ptx::grid_dep_launch();
+    ptx::grid_dep_wait();   // global memory from here on
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, 0);
@@ -240,10 +252,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::prefetch_tensormap(&map_ckv64);
             ptx::prefetch_tensormap(&map_kr32);
         }
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc<2>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
-        ptx::tmem_relinquish<2>();
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -365,6 +373,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         ptx::mma_commit_pair(bar(&misc->s_full[sb]), 0x3);
                         ++kq;
                         if (++tq == wq.t_end) {
+                            // the segment's last QK^T: once done, its Q may be replaced
+                            ptx::mma_commit_pair(bar(&misc->q_free), 0x3);
                             q_has = wq.next();
                             ++gq;
                             q_ready_seen = false;
@@ -433,8 +443,146 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::mma_commit_pair(bar(&misc->drain), 0x1);
             wait_bounded<false>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
         }
+    } else if (warp >= kSegWarp0) {
+        // ------------------------------------------------------ segment warps
+        // One warp per tensor-memory lane quadrant. At a segment's start they
+        // load its Q; when the last QK^T of a segment is done they load the next
+        // segment's Q, and when its last P.V is done they write its partial
+        // result -- so neither sits on the softmax warps' path from one tile to
+        // the next.
+        const int q4 = warp & 3;                       // TMEM lane quadrant
+        const int lt = q4 * 32 + lane;                 // TMEM lane 0..127
+        const int row = lt & 63;                       // local query row
+        const int half = lt >> 6;                      // which 128 channels of each MMA's 256
+        const int grow = ROWS_CTA * static_cast<int>(rank) + row;  // row within the sequence
+        const bool real_row = grow < args.rows;
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const int st_tid = threadIdx.x - kSegWarp0 * 32;   // 0..127
+        auto arrive_leader = [&](uint64_t *b) {
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) ptx::mbar_arrive(bar(b));
+                else ptx::mbar_arrive_cluster(leader_bar(b));
+            }
+        };
+        // Q of sequence b: channel blocks 0..5 into tensor memory in the
+        // duplicated 2-SM A layout (this lane holds row lt % 64, so lanes lt and
+        // lt ^ 64 carry the same row), blocks 6..8 into shared memory
+        // (128-byte swizzled, K-major).
+        // The loads are issued in three rounds of independent requests (the
+        // shared-memory blocks with the first round), so a segment start costs
+        // three global-load latencies rather than one per block.
+        auto load_q = [&](int32_t b) {
+            const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
+            const __nv_bfloat16 *qrow = qb + static_cast<int64_t>(real_row ? grow : 0) * D;
+            constexpr int NSM = ROWS_CTA * (NB - QT) * 8 / 128;   // 12 chunks of blocks 6..8 per thread
+            uint4 sv[NSM];
+#pragma unroll
+            for (int i = 0; i < NSM; ++i) {
+                const int idx = st_tid + 128 * i;
+                const int r = idx / ((NB - QT) * 8);
+                const int cc = idx - r * ((NB - QT) * 8);   // 16-byte chunk among blocks 6..8
+                const int gr = ROWS_CTA * static_cast<int>(rank) + r;
+                sv[i] = (gr < args.rows) ? ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + 64 * QT + cc * 8)
+                                         : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll 1
+            for (int j0 = 0; j0 < QT; j0 += 2) {   // two 64-channel blocks per round
+                uint4 v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    v[i] = real_row ? ld_global_nc_v4(qrow + 64 * j0 + 8 * i) : make_uint4(0, 0, 0, 0);
+                if (j0 == 0) {
+#pragma unroll
+                    for (int i = 0; i < NSM; ++i) {
+                        const int idx = st_tid + 128 * i;
+                        const int r = idx / ((NB - QT) * 8);
+                        const int cc = idx - r * ((NB - QT) * 8);
+                        st_shared_v4(base + OFF_Q + (cc >> 3) * (ROWS_CTA * 128) + sw128(r, cc & 7), sv[i].x,
+                                     sv[i].y, sv[i].z, sv[i].w);
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        w[4 * i] = v[8 * jj + i].x;
+                        w[4 * i + 1] = v[8 * jj + i].y;
+                        w[4 * i + 2] = v[8 * jj + i].z;
+                        w[4 * i + 3] = v[8 * jj + i].w;
+                    }
+                    ptx::tmem_st32(tmem + lane_base + TMEM_Q + 32 * (j0 + jj), w);
+                }
+            }
+            ptx::tmem_wait_st();
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            arrive_leader(&misc->q_ready);
+        };
+
+        auto prefetch_q = [&](int32_t b) {   // the next segment's Q rows into L2
+            if (!real_row || half) return;
+            const char *qrow = reinterpret_cast<const char *>(
+                args.q + (static_cast<int64_t>(b) * args.rows + grow) * D);
+#pragma unroll
+            for (int i = 0; i < D * 2 / 128; ++i)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128 * i));
+        };
+
+        int64_t k = 0;
+        int64_t g = 0;
+        bool have = walk.next();
+        if (have) load_q(walk.seg_b);
+        while (have && !*abort_flag) {
+            const int64_t slot = walk.slot;
+            const int64_t kl = k + (walk.t_end - walk.t_begin) - 1;   // the segment's last tile
+            k = kl + 1;
+            have = walk.next();
+            if (have) {
+                prefetch_q(walk.seg_b);
+                // the next segment's Q, once the last QK^T of this one is done
+                if (!wait_bounded<false>(bar(&misc->q_free), g & 1, abort_flag, args.timeout_ns)) break;
+                ptx::tc_fence_after();
+                load_q(walk.seg_b);
+            }
+            // this segment's partial result, once its last P.V is done
+            if (!wait_bounded<false>(bar(&misc->seg_done), g & 1, abort_flag, args.timeout_ns)) break;
+            if (!wait_bounded<false>(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
+                                     args.timeout_ns))
+                break;
+            ptx::tc_fence_after();
+            const float l_row = misc->seg_l[g & 1][row];
+            const float m_run = misc->seg_m[g & 1][row];
+            const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
+            float *dst = args.o_part + (slot * args.rows + grow) * DC;
+#pragma unroll 1
+            for (int cch = 0; cch < 8; ++cch) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
+                ptx::tmem_wait_ld();
+                if (real_row) {
+                    // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
+                    const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + ch);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv,
+                                            __uint_as_float(o[4 * j + 1]) * inv,
+                                            __uint_as_float(o[4 * j + 2]) * inv,
+                                            __uint_as_float(o[4 * j + 3]) * inv);
+                }
+            }
+            if (real_row && half == 0) {
+                args.lse_part[slot * args.rows + grow] =
+                    (l_row > 0.f) ? m_run * args.scale + logf(l_row) : -INFINITY;
+            }
+            ptx::tc_fence_before();
+            arrive_leader(&misc->o_free);
+            ++g;
+        }
     } else {
-        // ------------------------------------------------------ softmax / epilogue
+        // ------------------------------------------------------ softmax
         const int q4 = warp & 3;                       // TMEM lane quadrant
         const int lt = q4 * 32 + lane;                 // TMEM lane 0..127
         const int row = lt & 63;                       // local query row
@@ -451,47 +599,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 else ptx::mbar_arrive_cluster(leader_bar(b));
             }
         };
-        // Q of sequence b: channel blocks 0..5 into tensor memory in the
-        // duplicated 2-SM A layout (this lane holds row lt % 64, so lanes lt and
-        // lt ^ 64 carry the same row), blocks 6..8 into shared memory
-        // (128-byte swizzled, K-major).
-        auto load_q = [&](int32_t b) {
-            const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
-            const __nv_bfloat16 *qrow = qb + static_cast<int64_t>(real_row ? grow : 0) * D;
-#pragma unroll 1
-            for (int j = 0; j < QT; ++j) {
-                uint32_t w[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (real_row) v = ld_global_nc_v4(qrow + 64 * j + 8 * i);
-                    w[4 * i] = v.x;
-                    w[4 * i + 1] = v.y;
-                    w[4 * i + 2] = v.z;
-                    w[4 * i + 3] = v.w;
-                }
-                ptx::tmem_st32(tmem + lane_base + TMEM_Q + 32 * j, w);
-            }
-            for (int idx = st_tid; idx < ROWS_CTA * (NB - QT) * 8; idx += 128) {
-                const int r = idx / ((NB - QT) * 8);
-                const int cc = idx - r * ((NB - QT) * 8);   // 16-byte chunk among blocks 6..8
-                const int gr = ROWS_CTA * static_cast<int>(rank) + r;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (gr < args.rows)
-                    v = ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + 64 * QT + cc * 8);
-                const uint32_t dst = base + OFF_Q + (cc >> 3) * (ROWS_CTA * 128) + sw128(r, cc & 7);
-                st_shared_v4(dst, v.x, v.y, v.z, v.w);
-            }
-            ptx::tmem_wait_st();
-            ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            arrive_leader(&misc->q_ready);
-        };
-
         int64_t k = 0;
         int64_t seg_no = 0;
         bool have = walk.next();
-        if (have) load_q(walk.seg_b);
         while (have && !*abort_flag) {
             const int32_t seg_b = walk.seg_b;
             const int32_t L = walk.L;
@@ -611,17 +721,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
             if (!ok) break;
 
-            // next segment's Q may be loaded now: QK^T of this segment is complete
-            have = walk.next();
-            if (have) load_q(walk.seg_b);
-
-            // epilogue of this segment
-            const int64_t kl = k - 1;
-            if (!wait_bounded<false>(bar(&misc->pv_done[kl & 1]), (kl >> 1) & 1, abort_flag,
-                                     args.timeout_ns))
-                break;
-            ptx::tc_fence_after();
+            // the segment's row sum: both halves of the row meet; published with
+            // the running maximum for the segment warps' epilogue
             const uint32_t ltag = static_cast<uint32_t>(seg_no % 255) + 1u;
+            const int gpar = static_cast<int>(seg_no & 1);
             ++seg_no;
             const uint32_t lmine = (__float_as_uint(l_run) & 0xFFFFFF00u) | ltag;
             reinterpret_cast<volatile uint32_t *>(misc->xltag)[lt] = lmine;
@@ -629,32 +732,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (!wait_word(&misc->xltag[lt ^ 64], ltag, abort_flag, args.timeout_ns, &lother)) break;
             // identical in both lanes: the same two truncated terms, added commutatively
             const float l_row = __uint_as_float(lmine & 0xFFFFFF00u) + __uint_as_float(lother & 0xFFFFFF00u);
-            const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
-            float *dst = args.o_part + (slot * args.rows + grow) * DC;
-#pragma unroll 1
-            for (int cch = 0; cch < 8; ++cch) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
-                ptx::tmem_wait_ld();
-                if (real_row) {
-                    // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
-                    const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + ch);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv,
-                                            __uint_as_float(o[4 * j + 1]) * inv,
-                                            __uint_as_float(o[4 * j + 2]) * inv,
-                                            __uint_as_float(o[4 * j + 3]) * inv);
-                }
+            if (half == 0) {
+                misc->seg_l[gpar][row] = l_row;
+                misc->seg_m[gpar][row] = m_run;
             }
-            if (real_row && half == 0) {
-                args.lse_part[slot * args.rows + grow] =
-                    (l_row > 0.f) ? m_run * args.scale + logf(l_row) : -INFINITY;
-            }
-            ptx::tc_fence_before();
-            arrive_leader(&misc->o_free);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(&misc->seg_done));
             (void)seg_b;
+            (void)slot;
+            have = walk.next();
         }
     }
 
@@ -733,6 +819,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     for (uint32_t off = threadIdx.x * 16; off < OFF_MISC; off += kDecodeThreads * 16)
         st_shared_v4(base + off, 0, 0, 0, 0);
     ptx::fence_proxy_async_smem();
+    if (warp == 1) {
+        ptx::tmem_alloc<1>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
+        ptx::tmem_relinquish<1>();
+    }
+    ptx::grid_dep_launch();
+    ptx::grid_dep_wait();   // global memory from here on
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, 0);
@@ -748,10 +840,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             ptx::prefetch_tensormap(&map_ckv);
             ptx::prefetch_tensormap(&map_kr);
         }
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc<1>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
-        ptx::tmem_relinquish<1>();
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -893,17 +981,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(b));
         };
-        auto load_q = [&](int32_t b) {
+        auto load_q = [&](int32_t b) {   // all of a thread's loads in flight at once
             const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
-            for (int idx = st_tid; idx < ROWS * (D / 8); idx += 128) {
+            constexpr int NQ = ROWS * (D / 8) / 128;   // 9 chunks per thread
+            uint4 v[NQ];
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                const int idx = st_tid + 128 * i;
                 const int r = idx / (D / 8);
                 const int cc = idx - r * (D / 8);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (r < args.rows) v = ld_global_nc_v4(qb + static_cast<int64_t>(r) * D + cc * 8);
+                v[i] = (r < args.rows) ? ld_global_nc_v4(qb + static_cast<int64_t>(r) * D + cc * 8)
+                                       : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                const int idx = st_tid + 128 * i;
+                const int r = idx / (D / 8);
+                const int cc = idx - r * (D / 8);
                 uint32_t dst;
                 if (cc < 8) dst = base + OFF_Q + sw128(r, cc);
                 else dst = base + OFF_Q + Q_LAT + (r >> 3) * 128 + (r & 7) * 16;
-                st_shared_v4(dst, v.x, v.y, v.z, v.w);
+                st_shared_v4(dst, v[i].x, v[i].y, v[i].z, v[i].w);
             }
             ptx::fence_proxy_async_smem();
             arrive(&misc->q_ready);

@@ -142,6 +142,26 @@ mla_status pool_map(CUtensorMap *m, const mla_pool *pool, int32_t channels, int3
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the kernel before it on the stream finishes; it waits for that
+// kernel's completion (griddepcontrol.wait) before its first global-memory
+// access, so only its launch and on-chip set-up overlap.
+template <typename... KArgs, typename... Args>
+mla_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -188,8 +208,8 @@ mla_status launch_proj(const void *x, const void *w, void *out, const void *rope
     a.NT = NT;
     a.stages = std::min(mla::kProjStages, (K + 63) / 64);
     dim3 grid(H, (n_cols + 127) / 128, (T + NT - 1) / NT);
-    mla::proj_tc_kernel<<<grid, 128, mla::proj_smem_bytes(NT, a.stages), s>>>(mw, mx, a);
-    return launch_status();
+    return launch_pdl(mla::proj_tc_kernel, grid, dim3(128), mla::proj_smem_bytes(NT, a.stages), s, mw, mx,
+                      a);
 }
 
 mla_status check_pool(const mla_pool *p, int32_t channels) {
@@ -378,18 +398,17 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
         if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
             return st;
-        mla::decode_pair_kernel<<<2 * num_parts, mla::kPairThreads, mla::pair::SMEM_BYTES, s>>>(
-            m32, m64, mkr, a);
+        return launch_pdl(mla::decode_pair_kernel, dim3(2 * num_parts), dim3(mla::kPairThreads),
+                          mla::pair::SMEM_BYTES, s, m32, m64, mkr, a);
     } else {
         CUtensorMap mc, mkr;
         if ((st = pool_map(&mc, ckv, 64, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
             return st;
         if ((st = pool_map(&mkr, kr, 8, num_pages, 8, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != MLA_OK)
             return st;
-        mla::decode_single_kernel<<<num_parts, mla::kDecodeThreads, mla::single::SMEM_BYTES, s>>>(
-            mc, mkr, a);
+        return launch_pdl(mla::decode_single_kernel, dim3(num_parts), dim3(mla::kDecodeThreads),
+                          mla::single::SMEM_BYTES, s, mc, mkr, a);
     }
-    return launch_status();
 }
 
 mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t workspace_bytes,
@@ -422,8 +441,7 @@ mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t works
     a.tile_tokens = tile_tokens(variant_of(dims));
     a.num_parts = num_parts;
     dim3 grid(batch, static_cast<unsigned>((R + 3) / 4));
-    mla::combine_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_status();
+    return launch_pdl(mla::combine_kernel, grid, dim3(128), 0, static_cast<cudaStream_t>(stream), a);
 }
 
 mla_status mla_get_device_error(int32_t *code, void *stream) {
@@ -551,13 +569,15 @@ mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = mla::co_smem_bytes(KC, NT);
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(KS);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // as launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, mla::combine_out_kernel, mw, a) != cudaSuccess) return MLA_ERR_CUDA;
     return launch_status();
 }

@@ -28,6 +28,20 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it on the stream is still running. grid_dep_wait() blocks
+// until that kernel has completed and its memory writes are visible; every
+// such kernel here calls it before its first global-memory access.
+// grid_dep_launch() lets the next kernel on the stream be scheduled early.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- cluster
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

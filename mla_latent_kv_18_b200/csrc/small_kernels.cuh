@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
     __shared__ int64_t s_base, s_count;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t b = blockIdx.x;
+    ptx::grid_dep_launch();
+    ptx::grid_dep_wait();   // the partials come from the kernel before
     if (warp == 0) {
         int64_t base, cnt;
         sequence_slots(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts, b,
@@ -286,6 +288,8 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
         ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
         ptx::tmem_relinquish<1>();
     }
+    ptx::grid_dep_launch();
+    ptx::grid_dep_wait();   // global memory from here on
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -457,6 +461,8 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     uint32_t tcols = 32;
     while (tcols < static_cast<uint32_t>(NT)) tcols <<= 1;
 
+    ptx::grid_dep_launch();
+    ptx::grid_dep_wait();   // global memory from here on
     if (threadIdx.x == 0) {
         ptx::mbar_init(wfull, 1);
         ptx::mbar_init(done, 1);
