@@ -82,6 +82,19 @@ __device__ __forceinline__ uint4 ld_global_nc_v4(const void *p) {
     return v;
 }
 
+// Maximum of N values as eight interleaved chains and a tree (short
+// dependency depth; max is exact in any order).
+template <int N>
+__device__ __forceinline__ float max_of(const float (&v)[N]) {
+    static_assert(N % 8 == 0, "N");
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = v[i];
+#pragma unroll
+    for (int j = 8; j < N; ++j) m[j & 7] = fmaxf(m[j & 7], v[j]);
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
 // 128-byte-swizzled K-major block whose rows are 128 bytes apart.
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
@@ -626,12 +639,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
                 const int32_t tok0 = static_cast<int32_t>(t) * TOK + half * OWN;
                 float v[32];
-                float mx = -INFINITY;
+                if (tok0 + 32 <= vis) {   // every token of this half visible: no mask
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    v[j] = (tok0 + j < vis) ? __uint_as_float(sr[j]) : -INFINITY;
-                    mx = fmaxf(mx, v[j]);
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(sr[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = (tok0 + j < vis) ? __uint_as_float(sr[j]) : -INFINITY;
                 }
+                float mx = max_of<32>(v);
                 // half-row maxima meet through tagged words: low 8 mantissa bits
                 // carry the tile tag, both lanes use the same truncated values
                 const uint32_t tag = static_cast<uint32_t>((k >> 1) % 255) + 1u;
@@ -1042,12 +1057,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 float alpha = 1.f;
                 if (warp_real) {
                     const int32_t tok0 = static_cast<int32_t>(t) * TOK;
-                    float mx = -INFINITY;
+                    if (tok0 + TOK > vis) {   // mask the tokens this row does not see
 #pragma unroll
-                    for (int j = 0; j < TOK; ++j) {
-                        v[j] = (tok0 + j < vis) ? v[j] : -INFINITY;
-                        mx = fmaxf(mx, v[j]);
+                        for (int j = 0; j < TOK; ++j) v[j] = (tok0 + j < vis) ? v[j] : -INFINITY;
                     }
+                    const float mx = max_of<TOK>(v);
                     if (mx > -INFINITY && (m_run == -INFINITY ||
                                            (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
                         alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - mx) * args.scale_log2);
