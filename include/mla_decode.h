@@ -126,12 +126,16 @@ size_t mla_decode_workspace_size(const mla_dims *dims, int32_t batch, int32_t nu
 
 /*
  * Split-KV decode in latent space (the absorbed score and value steps).
- * The flattened list of tiles of all sequences (N tiles of 64 tokens for
- * d_latent 512, of 128 tokens for d_latent 64) is cut into P = min(num_parts, N)
- * contiguous ranges, range p holding tiles [floor(p N / P), floor((p+1) N / P));
- * each range is processed by one CTA pair (d_latent 512) or one CTA
- * (d_latent 64). For every (sequence, range) overlap it writes one slot of the
- * workspace, slots numbered sequence-major:
+ * The tiles of all sequences (N tiles of 64 tokens for d_latent 512, of 128
+ * tokens for d_latent 64) are laid end to end with W virtual tiles between
+ * consecutive non-empty sequences (W = 8 for 64-token tiles, 3 for 128-token
+ * tiles: the cost of switching to another sequence inside a range, a Q load
+ * and a partial-result write). The C = N + W (sequences - 1) positions are cut
+ * into P = min(num_parts, N) contiguous ranges, range p holding positions
+ * [floor(p C / P), floor((p+1) C / P)), and each range's real tiles are
+ * processed by one CTA pair (d_latent 512) or one CTA (d_latent 64); a range
+ * that lies inside a gap has none. For every (sequence, range) overlap it
+ * writes one slot of the workspace, slots numbered sequence-major:
  *   s[r, t]  = scale * (Q[b, r, 0:d_c] . c_KV[t] + Q[b, r, d_c:] . k_R[t])
  *   o[r, :]  = sum_t softmax(s[r, :])_t c_KV[t]       over the range's visible tokens
  *   lse[r]   = log sum_t exp(s[r, t])

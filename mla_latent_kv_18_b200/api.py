@@ -302,16 +302,45 @@ class Decoder:
         return self.out
 
 
+# (partition count, workspace) per (dims, batch, table width, tile total, device,
+# stream): decode() plans and allocates its workspace once per shape.
+_DECODE_PLANS = {}
+
+
+def _decode_plan(dims, batch, max_pages, total_tiles, device, stream):
+    key = (tuple(getattr(dims, f) for f, _ in dims._fields_), batch, max_pages, total_tiles,
+           torch.device(device), stream.cuda_stream)
+    plan = _DECODE_PLANS.get(key)
+    if plan is None:
+        parts = num_parts_for(dims, total_tiles, device)
+        plan = (parts, alloc_workspace(dims, batch, parts, device))
+        _DECODE_PLANS[key] = plan
+    return plan
+
+
 def decode(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, total_tiles=None,
            scale=0.0, stream=None):
-    """One decode step. Returns (out [B,n_q,H,d_v], o_lat [B,n_q,H,d_c], lse [B,n_q,H])."""
+    """One decode step. Returns (out [B,n_q,H,d_v], o_lat [B,n_q,H,d_c], lse [B,n_q,H]).
+
+    Serving-shaped: nothing is read back from the device. The partition count
+    comes from total_tiles when given (sum over sequences of ceil(L_b / tile)),
+    else from the block table's capacity (every sequence at max_pages pages);
+    the plan and the split-KV workspace are made once per (shape, stream) and
+    reused, and outputs come from PyTorch's caching allocator, so a warm call
+    does not allocate device memory. Calls on one stream reuse its workspace in
+    order; calls on different streams get different workspaces."""
     dims = dims_for(q_c, q_r, w_uk, w_uv, ckv_pool.shape[1], scale)
+    B, max_pages = block_table.shape
+    s = stream if stream is not None else torch.cuda.current_stream(q_c.device)
     if total_tiles is None:
         T = tile_tokens(dims)
-        total_tiles = int(((seq_lens.to(torch.int64) + T - 1) // T).sum().item())
-    dec = Decoder(dims, block_table.shape[0], block_table.shape[1], total_tiles, q_c.device)
-    out = dec(q_c, q_r, ckv_pool, kr_pool, block_table, seq_lens, w_uk, w_uv, stream=stream)
-    return out, dec.o_lat, dec.lse
+        total_tiles = B * ((max_pages * dims.page_size + T - 1) // T)
+    parts, ws = _decode_plan(dims, B, max_pages, int(total_tiles), q_c.device, s)
+    q = absorb_q(q_c, q_r, w_uk, dims, stream=s)
+    decode_splitkv(q, ckv_pool, kr_pool, block_table, seq_lens, dims, parts, workspace=ws, stream=s)
+    o_lat, lse = combine(ws, seq_lens, max_pages, dims, parts, stream=s)
+    out = absorb_out(o_lat, w_uv, dims, stream=s)
+    return out, o_lat, lse
 
 
 # ----------------------------------------------------------------------------

@@ -76,20 +76,30 @@ __device__ __forceinline__ bool wait_word(const uint32_t *slot, uint32_t tag,
 
 // ---------------------------------------------------------------------------
 // Partition plan. The tiles (tile_tokens tokens each) of all sequences are
-// laid end to end; partition p of P owns tiles [start(p), start(p+1)) with
-// start(p) = floor(p * N / P). A sequence b with n_b tiles starting at tile
-// offset O_b is covered by partitions part(O_b) .. part(O_b + n_b - 1) and
-// gets one partial slot per covering partition; slots are numbered
-// sequence-major.
+// laid end to end, and before every non-empty sequence but the first the plan
+// counts W = switch_cost(tile_tokens) virtual tiles: a partition that crosses
+// into another sequence pays a Q load and a partial-result write there, so it
+// gets correspondingly fewer real tiles. Sequence b, the j-th non-empty one,
+// occupies the cost range [C_b, C_b + n_b) with C_b = O_b + W j (O_b its first
+// tile); the total cost is C = N + W (NB - 1). Partition p of P owns the cost
+// range [start(p), start(p+1)), start(p) = floor(p * C / P), i.e. the tiles
+// whose cost position falls in it (a range inside a gap owns none). A sequence
+// is covered by partitions part(C_b) .. part(C_b + n_b - 1) and gets one
+// partial slot per covering partition; slots are numbered sequence-major.
+// With W = 0 this is an even split of the tiles.
 // ---------------------------------------------------------------------------
 
-__host__ __device__ __forceinline__ int64_t part_start(int64_t p, int64_t N, int64_t P) {
-    return (p * N) / P;
+__host__ __device__ __forceinline__ constexpr int32_t switch_cost(int32_t tile_tokens) {
+    return tile_tokens == 64 ? 8 : 3;
 }
 
-// Partition that owns tile t (0 <= t < N): the largest p with start(p) <= t.
-__host__ __device__ __forceinline__ int64_t part_of_tile(int64_t t, int64_t N, int64_t P) {
-    return ((t + 1) * P + N - 1) / N - 1;
+__host__ __device__ __forceinline__ int64_t part_start(int64_t p, int64_t C, int64_t P) {
+    return (p * C) / P;
+}
+
+// Partition that owns cost position c (0 <= c < C): the largest p with start(p) <= c.
+__host__ __device__ __forceinline__ int64_t part_of_tile(int64_t c, int64_t C, int64_t P) {
+    return ((c + 1) * P + C - 1) / C - 1;
 }
 
 // Usable length of sequence b and its tile count. Lengths outside
@@ -107,68 +117,78 @@ __host__ __device__ __forceinline__ int64_t tiles_of_len(int32_t L, int32_t tile
     return (static_cast<int64_t>(L) + tile_tokens - 1) / tile_tokens;
 }
 
+// Total plan cost from the tile total N and the number NB of non-empty sequences.
+__host__ __device__ __forceinline__ int64_t plan_cost(int64_t N, int64_t NB, int32_t tile_tokens) {
+    return N + static_cast<int64_t>(switch_cost(tile_tokens)) * (NB > 0 ? NB - 1 : 0);
+}
+
 struct SeqCursor {
     int32_t b;          // sequence index
-    int64_t tile_off;   // O_b
+    int64_t cost_off;   // C_b
     int64_t slot_base;  // S_b
-    int64_t total;      // N
-    int64_t parts;      // partitions in use: min(num_parts, N), so each owns >= 1 tile
+    int64_t total;      // C (plan cost; 0 when there is no tile)
+    int64_t parts;      // partitions in use: min(num_parts, N)
 };
 
 __host__ __device__ __forceinline__ int64_t parts_in_use(int64_t num_parts, int64_t N) {
     return N < num_parts ? N : num_parts;
 }
 
-// Warp-cooperative scan: the sequence whose tile range contains tile `ts`
-// (or the first sequence with a tile at or after ts), with its tile offset and
-// slot base. All 32 lanes must call it; every lane gets the result.
+// Warp-cooperative scan: the first non-empty sequence whose cost range ends
+// after cost position `ts` (the one a partition starting at ts begins with),
+// with its cost offset and slot base; ts < 0 asks only for the totals. All 32
+// lanes must call it; every lane gets the result.
 __device__ inline SeqCursor find_sequence(const int32_t *seq_lens, int32_t batch, int32_t max_pages,
                                           int32_t n_q, int32_t tile_tokens, int64_t P,
                                           int64_t ts) {
     const int lane = threadIdx.x & 31;
+    const int64_t W = switch_cost(tile_tokens);
     bool bad = false;
-    int64_t N = 0;
+    int64_t N = 0, NB = 0;
     for (int32_t base = 0; base < batch; base += 32) {
         int32_t b = base + lane;
         int64_t n = 0;
         if (b < batch) n = tiles_of_len(clamp_len(seq_lens[b], max_pages, n_q, &bad), tile_tokens);
-        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-        N += n;
+        N += __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(n));
+        NB += __popc(__ballot_sync(0xffffffffu, n > 0));
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(kErrDeviceBounds);
-    SeqCursor cur{batch, N, 0, N, parts_in_use(P, N)};
-    if (N == 0) return cur;
+    const int64_t C = plan_cost(N, NB, tile_tokens);
+    SeqCursor cur{batch, C, 0, C, parts_in_use(P, N)};
+    if (N == 0 || ts < 0) return cur;
     P = cur.parts;
-    int64_t O = 0, S = 0;
+    int64_t CO = 0, S = 0;
     for (int32_t base = 0; base < batch; base += 32) {
         int32_t b = base + lane;
         int64_t n = 0;
         if (b < batch) n = tiles_of_len(clamp_len(seq_lens[b], max_pages, n_q, &bad), tile_tokens);
-        // exclusive prefix of n across the warp
-        int64_t incl = n;
+        // each non-empty sequence costs its tiles plus the gap after it, so the
+        // exclusive prefix of that cost is C_b
+        const int64_t w = (n > 0) ? n + W : 0;
+        int64_t incl = w;
         for (int o = 1; o < 32; o <<= 1) {
             int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        const int64_t Ob = O + incl - n;
+        const int64_t Cb = CO + incl - w;
         int64_t ns = 0;
-        if (n > 0) ns = part_of_tile(Ob + n - 1, N, P) - part_of_tile(Ob, N, P) + 1;
+        if (n > 0) ns = part_of_tile(Cb + n - 1, C, P) - part_of_tile(Cb, C, P) + 1;
         int64_t sincl = ns;
         for (int o = 1; o < 32; o <<= 1) {
             int64_t v = __shfl_up_sync(0xffffffffu, sincl, o);
             if (lane >= o) sincl += v;
         }
         const int64_t Sb = S + sincl - ns;
-        const bool hit = (n > 0) && (Ob + n > ts);
+        const bool hit = (n > 0) && (Cb + n > ts);
         const unsigned m = __ballot_sync(0xffffffffu, hit);
         if (m) {
             const int src = __ffs(m) - 1;
             cur.b = __shfl_sync(0xffffffffu, b, src);
-            cur.tile_off = __shfl_sync(0xffffffffu, Ob, src);
+            cur.cost_off = __shfl_sync(0xffffffffu, Cb, src);
             cur.slot_base = __shfl_sync(0xffffffffu, Sb, src);
             return cur;
         }
-        O += __shfl_sync(0xffffffffu, incl, 31);
+        CO += __shfl_sync(0xffffffffu, incl, 31);
         S += __shfl_sync(0xffffffffu, sincl, 31);
     }
     return cur;

@@ -74,6 +74,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint4 ld_global_nc_v4(const void *p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -101,15 +110,16 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
-// Iterates the (sequence, tile range) segments of one partition. Every thread
-// that walks it gets the same sequence of segments.
+// Iterates the (sequence, tile range) segments of one partition: the tiles
+// whose plan cost position falls in [tile, te). Every thread that walks it gets
+// the same sequence of segments.
 struct SegmentWalker {
     const int32_t *seq_lens;
     int32_t batch, max_pages, n_q, tile_tokens;
-    int64_t N, P, p, te;
+    int64_t N, P, p, te;   // N: plan cost C; te: end of this partition's cost range
     // current state
     int32_t b;
-    int64_t O, S, tile;
+    int64_t O, S, tile;    // O: cost offset C_b of sequence b; tile: cost position reached
     // current segment
     int32_t seg_b, L;
     int64_t t_begin, t_end, slot;
@@ -120,16 +130,17 @@ struct SegmentWalker {
             const int32_t Lb = clamp_len(seq_lens[b], max_pages, n_q, &bad);
             const int64_t n = tiles_of_len(Lb, tile_tokens);
             if (n == 0) { ++b; continue; }
+            if (O >= te) return false;   // the next sequence starts past this partition
             const int64_t pf = part_of_tile(O, N, P);
             seg_b = b;
             L = Lb;
-            t_begin = tile - O;
+            t_begin = (tile > O) ? tile - O : 0;
             t_end = (te - O < n) ? (te - O) : n;
             slot = S + (p - pf);
             tile = O + t_end;
             const int64_t pl = part_of_tile(O + n - 1, N, P);
             S += pl - pf + 1;
-            O += n;
+            O += n + switch_cost(tile_tokens);
             ++b;
             return true;
         }
@@ -159,7 +170,9 @@ constexpr uint32_t OFF_PV = OFF_QK + QK_STAGES * STAGE_QK;  // P.V ring
 constexpr uint32_t OFF_P = OFF_PV + PV_STAGES * STAGE_PV;
 constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 217088
 constexpr uint32_t MISC_BYTES = 3072;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES;   // dynamic smem base is 1 KB aligned
+constexpr uint32_t OFF_EPI = OFF_MISC + MISC_BYTES;         // partial-store staging, 2 KB per segment warp
+constexpr uint32_t EPI_BYTES = 4 * 32 * 64;
+constexpr uint32_t SMEM_BYTES = OFF_EPI + EPI_BYTES;     // dynamic smem base is 1 KB aligned
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
 constexpr uint32_t TMEM_S = 256;               // two 32-column score buffers
@@ -183,7 +196,7 @@ struct Misc {
     int32_t abort_flag;
     int32_t cur_b;
     int32_t pad0;
-    int64_t cur_O, cur_S, cur_N;
+    int64_t cur_O, cur_S, cur_N, cur_P;   // plan: cost offset, slot base, total cost, partitions
     uint32_t xtag[2][128];            // pair kernel: tagged half-row maxima, by tile parity
     uint32_t xltag[128];              // pair kernel: tagged half-row sums, per segment
     uint64_t q_free;                  // pair kernel: the last QK^T of a segment is done (Q may be replaced)
@@ -251,16 +264,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     ptx::grid_dep_wait();   // global memory from here on
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
-                                          P, 0);
-        const int64_t N = c.total;
+                                          P, -1);
+        const int64_t N = c.total;   // plan cost
         const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
         const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, ts);
         if (lane == 0) {
             misc->cur_b = s.b;
-            misc->cur_O = s.tile_off;
+            misc->cur_O = s.cost_off;
             misc->cur_S = s.slot_base;
             misc->cur_N = N;
+            misc->cur_P = c.parts;
             ptx::prefetch_tensormap(&map_ckv32);
             ptx::prefetch_tensormap(&map_ckv64);
             ptx::prefetch_tensormap(&map_kr32);
@@ -279,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     walk.n_q = args.n_q;
     walk.tile_tokens = TOK;
     walk.N = misc->cur_N;
-    walk.P = parts_in_use(P, walk.N);
+    walk.P = misc->cur_P;
     walk.p = part;
     walk.b = misc->cur_b;
     walk.O = misc->cur_O;
@@ -568,22 +582,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const float l_row = misc->seg_l[g & 1][row];
             const float m_run = misc->seg_m[g & 1][row];
             const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
-            float *dst = args.o_part + (slot * args.rows + grow) * DC;
+            // O / l of this lane's row, 16 columns at a time through a 2 KB
+            // shared-memory tile ([32 rows x 64 B], 16-byte chunks XOR-swizzled
+            // by row), so that each global store instruction writes 8 rows x 64
+            // contiguous bytes instead of 32 rows x 16 bytes
+            const uint32_t stg = base + OFF_EPI + static_cast<uint32_t>(warp - kSegWarp0) * 2048u;
+            const int rr = lane >> 2, rc = lane & 3;   // read-back: rows rr + 8i, chunk rc
 #pragma unroll 1
             for (int cch = 0; cch < 8; ++cch) {
                 uint32_t o[32];
                 ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
                 ptx::tmem_wait_ld();
-                if (real_row) {
-                    // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
-                    const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + ch);
+                // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
+                const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv,
-                                            __uint_as_float(o[4 * j + 1]) * inv,
-                                            __uint_as_float(o[4 * j + 2]) * inv,
-                                            __uint_as_float(o[4 * j + 3]) * inv);
+                for (int pc = 0; pc < 2; ++pc) {
+                    __syncwarp();   // the previous piece has been read back
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int j = 16 * pc + 4 * c;
+                        st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4),
+                                     __float_as_uint(__uint_as_float(o[j]) * inv),
+                                     __float_as_uint(__uint_as_float(o[j + 1]) * inv),
+                                     __float_as_uint(__uint_as_float(o[j + 2]) * inv),
+                                     __float_as_uint(__uint_as_float(o[j + 3]) * inv));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = rr + 8 * i;                         // staging row = lane r of this warp
+                        const int grow_r = ROWS_CTA * static_cast<int>(rank) + ((q4 * 32 + r) & 63);
+                        const uint4 v = ld_shared_v4(stg + r * 64 + ((rc ^ ((r >> 1) & 3)) << 4));
+                        if (grow_r < args.rows)
+                            *reinterpret_cast<uint4 *>(args.o_part + (slot * args.rows + grow_r) * DC + ch +
+                                                       16 * pc + 4 * rc) = v;
+                    }
                 }
             }
             if (real_row && half == 0) {
@@ -842,16 +875,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     ptx::grid_dep_wait();   // global memory from here on
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
-                                          P, 0);
-        const int64_t N = c.total;
+                                          P, -1);
+        const int64_t N = c.total;   // plan cost
         const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
         const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, ts);
         if (lane == 0) {
             misc->cur_b = s.b;
-            misc->cur_O = s.tile_off;
+            misc->cur_O = s.cost_off;
             misc->cur_S = s.slot_base;
             misc->cur_N = N;
+            misc->cur_P = c.parts;
             ptx::prefetch_tensormap(&map_ckv);
             ptx::prefetch_tensormap(&map_kr);
         }
@@ -868,7 +902,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     walk.n_q = args.n_q;
     walk.tile_tokens = TOK;
     walk.N = misc->cur_N;
-    walk.P = parts_in_use(P, walk.N);
+    walk.P = misc->cur_P;
     walk.p = part;
     walk.b = misc->cur_b;
     walk.O = misc->cur_O;

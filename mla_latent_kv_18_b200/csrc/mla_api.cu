@@ -100,6 +100,22 @@ mla_status device_ready() {
             st.status = MLA_ERR_CUDA;
             return;
         }
+        // The decode step's kernels keep the same (largest) shared-memory
+        // carve-out, so an SM does not reconfigure between them.
+        const int carve = cudaSharedmemCarveoutMaxShared;
+        if (cudaFuncSetAttribute(mla::proj_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(mla::combine_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carve) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_pair_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carve) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_single_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carve) != cudaSuccess) {
+            st.status = MLA_ERR_CUDA;
+            return;
+        }
     });
     return st.status;
 }
@@ -275,25 +291,30 @@ int64_t mla_decode_plan(const mla_dims *dims, const int32_t *seq_lens_host,
         return -1;
     if (batch > 0 && !seq_lens_host) return -1;
     const int T = tile_tokens(variant_of(dims));
-    int64_t N = 0;
+    int64_t N = 0, NB = 0;
     bool bad = false;
-    for (int32_t b = 0; b < batch; ++b)
-        N += mla::tiles_of_len(mla::clamp_len(seq_lens_host[b], max_pages_per_seq, dims->n_q, &bad), T);
+    for (int32_t b = 0; b < batch; ++b) {
+        const int64_t n =
+            mla::tiles_of_len(mla::clamp_len(seq_lens_host[b], max_pages_per_seq, dims->n_q, &bad), T);
+        N += n;
+        NB += (n > 0);
+    }
+    const int64_t C = mla::plan_cost(N, NB, T);
     const int64_t P = mla::parts_in_use(num_parts, N);
-    int64_t O = 0, S = 0;
+    int64_t CO = 0, S = 0;   // cost offset of the next non-empty sequence, slots so far
     for (int32_t b = 0; b < batch; ++b) {
         const int64_t n =
             mla::tiles_of_len(mla::clamp_len(seq_lens_host[b], max_pages_per_seq, dims->n_q, &bad), T);
         int64_t pf = -1, cnt = 0;
         if (n > 0) {
-            pf = mla::part_of_tile(O, N, P);
-            cnt = mla::part_of_tile(O + n - 1, N, P) - pf + 1;
+            pf = mla::part_of_tile(CO, C, P);
+            cnt = mla::part_of_tile(CO + n - 1, C, P) - pf + 1;
+            CO += n + mla::switch_cost(T);
         }
         if (part_first) part_first[b] = static_cast<int32_t>(pf);
         if (slot_count) slot_count[b] = static_cast<int32_t>(cnt);
         if (slot_base) slot_base[b] = S;
         S += cnt;
-        O += n;
     }
     return S;
 }

@@ -12,38 +12,43 @@
 
 namespace mla {
 
-// (slot_base, slot_count) of sequence b under the partition plan; warp-wide.
+// (slot_base, slot_count) of sequence b under the partition plan (the
+// cost-weighted split of common.cuh); warp-wide.
 __device__ inline void sequence_slots(const int32_t *seq_lens, int32_t batch, int32_t max_pages,
                                       int32_t n_q, int32_t tile_tokens, int64_t P, int32_t b,
                                       int64_t *slot_base, int64_t *slot_count) {
     const int lane = threadIdx.x & 31;
+    const int64_t W = switch_cost(tile_tokens);
     bool bad = false;
-    int64_t N = 0;
+    int64_t N = 0, NB = 0;
     for (int32_t b0 = 0; b0 < batch; b0 += 32) {
         const int32_t bb = b0 + lane;
         int64_t n = 0;
         if (bb < batch) n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        NB += __popc(__ballot_sync(0xffffffffu, n > 0));
         for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
         N += n;
     }
-    int64_t O = 0, S = 0;
+    int64_t CO = 0, S = 0;
     *slot_base = 0;
     *slot_count = 0;
     if (N == 0) return;
+    const int64_t C = plan_cost(N, NB, tile_tokens);
     P = parts_in_use(P, N);
     for (int32_t b0 = 0; b0 <= b; b0 += 32) {
         const int32_t bb = b0 + lane;
         int64_t n = 0;
         if (bb < batch && bb <= b)
             n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
-        int64_t incl = n;
+        const int64_t w = (n > 0) ? n + W : 0;   // tiles plus the gap after the sequence
+        int64_t incl = w;
         for (int o = 1; o < 32; o <<= 1) {
             const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        const int64_t Ob = O + incl - n;
+        const int64_t Cb = CO + incl - w;
         int64_t ns = 0;
-        if (n > 0) ns = part_of_tile(Ob + n - 1, N, P) - part_of_tile(Ob, N, P) + 1;
+        if (n > 0) ns = part_of_tile(Cb + n - 1, C, P) - part_of_tile(Cb, C, P) + 1;
         int64_t sincl = ns;
         for (int o = 1; o < 32; o <<= 1) {
             const int64_t v = __shfl_up_sync(0xffffffffu, sincl, o);
@@ -55,7 +60,7 @@ __device__ inline void sequence_slots(const int32_t *seq_lens, int32_t batch, in
             *slot_count = __shfl_sync(0xffffffffu, ns, src);
             return;
         }
-        O += __shfl_sync(0xffffffffu, incl, 31);
+        CO += __shfl_sync(0xffffffffu, incl, 31);
         S += __shfl_sync(0xffffffffu, sincl, 31);
     }
 }
@@ -66,8 +71,9 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
                                             int32_t n_q, int32_t tile_tokens, int64_t P, int32_t b_lo,
                                             int32_t b_hi, int64_t *base, int32_t *cnt) {
     const int lane = threadIdx.x & 31;
+    const int64_t W = switch_cost(tile_tokens);
     bool bad = false;
-    int64_t N = 0;
+    int64_t N = 0, NB = 0;
     constexpr int kCached = 8;   // per-lane tile counts kept for the second pass (batch <= 256)
     int64_t nc[kCached];
 #pragma unroll
@@ -79,6 +85,7 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
     for (int c = 0; c < kCached; ++c) {
         if (32 * c >= batch) break;   // uniform over the warp
         int64_t n = nc[c];
+        NB += __popc(__ballot_sync(0xffffffffu, n > 0));
         for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
         N += n;
     }
@@ -86,6 +93,7 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
         const int32_t bb = b0 + lane;
         int64_t n = 0;
         if (bb < batch) n = tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
+        NB += __popc(__ballot_sync(0xffffffffu, n > 0));
         for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
         N += n;
     }
@@ -94,8 +102,9 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
         cnt[b - b_lo] = 0;
     }
     if (N == 0) return;
+    const int64_t C = plan_cost(N, NB, tile_tokens);
     P = parts_in_use(P, N);
-    int64_t O = 0, S = 0;
+    int64_t CO = 0, S = 0;
     for (int32_t b0 = 0; b0 <= b_hi; b0 += 32) {
         const int32_t bb = b0 + lane;
         int64_t n = 0;
@@ -107,14 +116,15 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
             n = cached >= 0 ? cached
                             : tiles_of_len(clamp_len(seq_lens[bb], max_pages, n_q, &bad), tile_tokens);
         }
-        int64_t incl = n;
+        const int64_t w = (n > 0) ? n + W : 0;   // tiles plus the gap after the sequence
+        int64_t incl = w;
         for (int o = 1; o < 32; o <<= 1) {
             const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        const int64_t Ob = O + incl - n;
+        const int64_t Cb = CO + incl - w;
         int64_t ns = 0;
-        if (n > 0) ns = part_of_tile(Ob + n - 1, N, P) - part_of_tile(Ob, N, P) + 1;
+        if (n > 0) ns = part_of_tile(Cb + n - 1, C, P) - part_of_tile(Cb, C, P) + 1;
         int64_t sincl = ns;
         for (int o = 1; o < 32; o <<= 1) {
             const int64_t v = __shfl_up_sync(0xffffffffu, sincl, o);
@@ -124,7 +134,7 @@ __device__ inline void sequence_slots_range(const int32_t *seq_lens, int32_t bat
             base[bb - b_lo] = S + sincl - ns;
             cnt[bb - b_lo] = static_cast<int32_t>(ns);
         }
-        O += __shfl_sync(0xffffffffu, incl, 31);
+        CO += __shfl_sync(0xffffffffu, incl, 31);
         S += __shfl_sync(0xffffffffu, sincl, 31);
     }
 }

@@ -53,26 +53,44 @@ def _dims(b, **kw):
     return b.MLADims(**d)
 
 
+# Virtual tiles the plan charges for each switch to another sequence inside a
+# partition (a Q load and a partial-result write): 8 for 64-token tiles, 3 for
+# 128-token tiles.
+SWITCH_COST = {64: 8, 128: 3}
+
+
 def _brute_plan(lens, max_pages, n_q, T, P):
+    """The partition plan by enumeration: lay the tiles of the non-empty sequences
+    end to end with SWITCH_COST[T] virtual positions between consecutive ones,
+    cut the positions into P nearly equal ranges, and count for each sequence
+    the ranges its real tiles fall in."""
     n = []
     for L in lens:
         L = max(0, min(L, max_pages * 64))
         n.append((L + T - 1) // T)
     N = sum(n)
     P = min(P, N) if N else P
-    owner = []
+    pos, seq_of_pos = 0, []           # cost position -> sequence (None for a virtual one)
+    for b, nb in enumerate(n):
+        if nb == 0:
+            continue
+        if seq_of_pos:
+            seq_of_pos += [None] * SWITCH_COST[T]
+        seq_of_pos += [b] * nb
+    C = len(seq_of_pos)
+    parts_of = [set() for _ in n]
     for p in range(P):
-        owner += [p] * ((p + 1) * N // P - p * N // P)
-    assert len(owner) == N
-    off, base = 0, 0
+        for c in range(p * C // P, (p + 1) * C // P):
+            if seq_of_pos[c] is not None:
+                parts_of[seq_of_pos[c]].add(p)
+    base = 0
     first, count, bases = [], [], []
-    for nb in n:
-        parts = sorted(set(owner[off:off + nb]))
+    for b in range(len(n)):
+        parts = sorted(parts_of[b])
         first.append(parts[0] if parts else -1)
         count.append(len(parts))
         bases.append(base)
         base += len(parts)
-        off += nb
     return first, count, bases, base
 
 

@@ -191,6 +191,10 @@ def test_partials_match_oracle_windows(api, name, parts):
     n_tiles = [(L + T - 1) // T for L in lens]
     N = sum(n_tiles)
     P = min(parts, N)
+    # the plan's cost positions: tiles end to end, SWITCH_COST[T] virtual positions
+    # between consecutive non-empty sequences; partition p owns [p C / P, (p+1) C / P)
+    W = {64: 8, 128: 3}[T]
+    C = N + W * (sum(1 for n in n_tiles if n) - 1)
     scale = oracle.default_scale(w.d_nope, w.d_rope)
     off = 0
     for b in range(w.batch):
@@ -198,8 +202,8 @@ def test_partials_match_oracle_windows(api, name, parts):
                for k, v in inp.items()}
         for j in range(int(cnt[b])):
             p = int(pf[b]) + j
-            t0 = max(p * N // P, off) - off
-            t1 = min((p + 1) * N // P, off + n_tiles[b]) - off
+            t0 = max(p * C // P, off) - off
+            t1 = min((p + 1) * C // P, off + n_tiles[b]) - off
             o_ref, lse_ref = oracle.attend_latent(r["q"][b:b + 1].cpu(), one["ckv_pool"],
                                                   one["kr_pool"], one["block_table"],
                                                   one["seq_lens"], scale, t_lo=t0 * T,
@@ -207,7 +211,7 @@ def test_partials_match_oracle_windows(api, name, parts):
             slot = int(base[b]) + j
             _check(o_part[slot].reshape(1, w.n_q, w.heads, -1), o_ref, f"slot {slot}")
             np.testing.assert_allclose(lse_part[slot].reshape(lse_ref.shape), lse_ref, atol=1e-3)
-        off += n_tiles[b]
+        off += n_tiles[b] + (W if n_tiles[b] else 0)
 
 
 @pytest.mark.parametrize("name,parts", [("dsv3", None), ("dsv3", 1), ("dsv3", 74),
