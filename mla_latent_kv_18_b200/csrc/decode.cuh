@@ -157,8 +157,9 @@ constexpr int NB = D / 64;                    // 9 K-blocks of 64 channels
 constexpr int ROWS_CTA = 64;                  // query rows per SM
 constexpr int TOK = 64;                       // tokens per tile (one page)
 constexpr int OWN = 32;                       // tokens per SM in QK^T
-constexpr int QT = 6;                         // Q channel blocks 0..5 live in tensor memory
-constexpr uint32_t Q_BYTES = (NB - QT) * ROWS_CTA * 128;    // 24576: Q blocks 6..8
+constexpr int QT = 5;                         // Q channel blocks 0..4 live in tensor memory
+constexpr int NSB = 3;                        // score buffers in tensor memory
+constexpr uint32_t Q_BYTES = (NB - QT) * ROWS_CTA * 128;    // 32768: Q blocks 5..8
 constexpr uint32_t STAGE_QK = NB * OWN * 128;               // 36864: own 32 tokens x 9 blocks
 constexpr uint32_t STAGE_PV = 4 * TOK * 128;                // 32768: 64 tokens x this SM's 4 blocks
 constexpr int QK_STAGES = 3;                                // QK^T ring depth
@@ -170,13 +171,13 @@ constexpr uint32_t OFF_PV = OFF_QK + QK_STAGES * STAGE_QK;  // P.V ring
 constexpr uint32_t OFF_P = OFF_PV + PV_STAGES * STAGE_PV;
 constexpr uint32_t OFF_MISC = OFF_P + 2 * P_BYTES;          // 217088
 constexpr uint32_t MISC_BYTES = 3072;
-constexpr uint32_t OFF_EPI = OFF_MISC + MISC_BYTES;         // partial-store staging, 2 KB per segment warp
-constexpr uint32_t EPI_BYTES = 4 * 32 * 64;
+constexpr uint32_t OFF_EPI = OFF_MISC + MISC_BYTES;         // partial-store staging, 1 KB per segment warp
+constexpr uint32_t EPI_BYTES = 4 * 32 * 32;
 constexpr uint32_t SMEM_BYTES = OFF_EPI + EPI_BYTES;     // dynamic smem base is 1 KB aligned
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
-constexpr uint32_t TMEM_S = 256;               // two 32-column score buffers
-constexpr uint32_t TMEM_Q = 320;               // Q blocks 0..5: 32 columns each (two bf16 per column)
+constexpr uint32_t TMEM_S = 256;               // three 32-column score buffers
+constexpr uint32_t TMEM_Q = TMEM_S + NSB * 32; // Q blocks 0..4: 32 columns each (two bf16 per column)
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, 256, 0, 1);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -187,7 +188,7 @@ static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 
 
 // misc-region layout (both kernels)
 struct Misc {
-    uint64_t full[2], empty[2], s_full[2], s_free[2], p_ready[2], pv_done[2], q_ready, o_free;
+    uint64_t full[2], empty[2], s_full[pair::NSB], s_free[2], p_ready[2], pv_done[2], q_ready, o_free;
     uint64_t drain;                   // MMA drain before tensor memory is freed
     uint64_t qk_full[pair::QK_STAGES], qk_empty[pair::QK_STAGES];   // the pair kernel's two rings
     uint64_t pv_full[pair::PV_STAGES], pv_empty[pair::PV_STAGES];
@@ -241,8 +242,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
             ptx::mbar_init(bar(&misc->pv_landed[i]), 1);
         }
+        for (int i = 0; i < NSB; ++i) ptx::mbar_init(bar(&misc->s_full[i]), 1);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(bar(&misc->s_full[i]), 1);
             ptx::mbar_init(bar(&misc->p_ready[i]), 8);
             ptx::mbar_init(bar(&misc->pv_done[i]), 1);
         }
@@ -355,8 +356,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer (leader)
-        // Two cursors: QK^T of tile kq and P.V of tile kp (kp < kq <= kp + 2,
-        // two score buffers). Whichever is ready is issued; the polls are
+        // Two cursors: QK^T of tile kq and P.V of tile kp (kp < kq <= kp + 3,
+        // three score buffers). Whichever is ready is issued; the polls are
         // non-blocking so a late KV tile never holds back a ready P.V.
         if (rank == 0 && ptx::elect_one()) {
             SegmentWalker wq = walk, wp = walk;
@@ -369,10 +370,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             uint32_t spins = 0;
             while ((q_has || p_has) && !*abort_flag) {
                 bool progressed = false;
-                if (q_has && kq < kp + 2) {
+                if (q_has && kq < kp + NSB) {
                     if (!q_ready_seen) q_ready_seen = ptx::mbar_test_wait(bar(&misc->q_ready), gq & 1);
                     const int s = static_cast<int>(kq % QK_STAGES);
-                    const int sb = static_cast<int>(kq & 1);
+                    const int sb = static_cast<int>(kq % NSB);   // score buffer: tile kq - 3's
+                                                                  // P.V is issued (its softmax read it)
                     if (q_ready_seen &&
                         ptx::mbar_test_wait(bar(&misc->qk_full[s]), (kq / QK_STAGES) & 1)) {
                         ptx::tc_fence_after();
@@ -414,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const bool first = (tp == wp.t_begin);
                     if (first && gp > 0 && !o_free_seen)
                         o_free_seen = ptx::mbar_test_wait(bar(&misc->o_free), (gp - 1) & 1);
-                    const int s = static_cast<int>(kp & 1);            // P buffer, score buffer
+                    const int s = static_cast<int>(kp & 1);            // P buffer
                     const int ps = static_cast<int>(kp % PV_STAGES);   // P.V operand slot
                     // Once both CTAs' copies of slot ps have landed, say so to each
                     // CTA: the softmax warps clear the rows past a sequence's end in
@@ -496,33 +498,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // duplicated 2-SM A layout (this lane holds row lt % 64, so lanes lt and
         // lt ^ 64 carry the same row), blocks 6..8 into shared memory
         // (128-byte swizzled, K-major).
-        // The loads are issued in three rounds of independent requests (the
-        // shared-memory blocks with the first round), so a segment start costs
-        // three global-load latencies rather than one per block.
+        // The loads are issued in three rounds of independent requests (half of
+        // the shared-memory blocks with each of the first two), so a segment
+        // start costs three global-load latencies rather than one per block.
         auto load_q = [&](int32_t b) {
             const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
             const __nv_bfloat16 *qrow = qb + static_cast<int64_t>(real_row ? grow : 0) * D;
-            constexpr int NSM = ROWS_CTA * (NB - QT) * 8 / 128;   // 12 chunks of blocks 6..8 per thread
-            uint4 sv[NSM];
-#pragma unroll
-            for (int i = 0; i < NSM; ++i) {
-                const int idx = st_tid + 128 * i;
-                const int r = idx / ((NB - QT) * 8);
-                const int cc = idx - r * ((NB - QT) * 8);   // 16-byte chunk among blocks 6..8
-                const int gr = ROWS_CTA * static_cast<int>(rank) + r;
-                sv[i] = (gr < args.rows) ? ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + 64 * QT + cc * 8)
-                                         : make_uint4(0, 0, 0, 0);
-            }
+            constexpr int NSM = ROWS_CTA * (NB - QT) * 8 / 128 / 2;   // 8 + 8 chunks of blocks 5..8
 #pragma unroll 1
-            for (int j0 = 0; j0 < QT; j0 += 2) {   // two 64-channel blocks per round
-                uint4 v[16];
+            for (int j0 = 0; j0 < QT; j0 += 2) {   // up to two 64-channel blocks per round
+                const int nj = (j0 + 1 < QT) ? 2 : 1;
+                uint4 v[16], sv[NSM];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    v[i] = real_row ? ld_global_nc_v4(qrow + 64 * j0 + 8 * i) : make_uint4(0, 0, 0, 0);
-                if (j0 == 0) {
+                    v[i] = (real_row && (i < 8 || nj == 2)) ? ld_global_nc_v4(qrow + 64 * j0 + 8 * i)
+                                                            : make_uint4(0, 0, 0, 0);
+                if (j0 < 4) {
 #pragma unroll
                     for (int i = 0; i < NSM; ++i) {
-                        const int idx = st_tid + 128 * i;
+                        const int idx = st_tid + 128 * (i + NSM * (j0 >> 1));
+                        const int r = idx / ((NB - QT) * 8);
+                        const int cc = idx - r * ((NB - QT) * 8);   // 16-byte chunk among blocks 5..8
+                        const int gr = ROWS_CTA * static_cast<int>(rank) + r;
+                        sv[i] = (gr < args.rows)
+                                    ? ld_global_nc_v4(qb + static_cast<int64_t>(gr) * D + 64 * QT + cc * 8)
+                                    : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int i = 0; i < NSM; ++i) {
+                        const int idx = st_tid + 128 * (i + NSM * (j0 >> 1));
                         const int r = idx / ((NB - QT) * 8);
                         const int cc = idx - r * ((NB - QT) * 8);
                         st_shared_v4(base + OFF_Q + (cc >> 3) * (ROWS_CTA * 128) + sw128(r, cc & 7), sv[i].x,
@@ -531,6 +535,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 }
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
+                    if (jj >= nj) break;
                     uint32_t w[32];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -582,12 +587,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const float l_row = misc->seg_l[g & 1][row];
             const float m_run = misc->seg_m[g & 1][row];
             const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
-            // O / l of this lane's row, 16 columns at a time through a 2 KB
-            // shared-memory tile ([32 rows x 64 B], 16-byte chunks XOR-swizzled
-            // by row), so that each global store instruction writes 8 rows x 64
+            // O / l of this lane's row, 8 columns at a time through a 1 KB
+            // shared-memory tile ([32 rows x 32 B], 16-byte chunks XOR-swizzled
+            // by row), so that each global store instruction writes 16 rows x 32
             // contiguous bytes instead of 32 rows x 16 bytes
-            const uint32_t stg = base + OFF_EPI + static_cast<uint32_t>(warp - kSegWarp0) * 2048u;
-            const int rr = lane >> 2, rc = lane & 3;   // read-back: rows rr + 8i, chunk rc
+            const uint32_t stg = base + OFF_EPI + static_cast<uint32_t>(warp - kSegWarp0) * 1024u;
+            const int rr = lane >> 1, rc = lane & 1;   // read-back: rows rr + 16i, chunk rc
 #pragma unroll 1
             for (int cch = 0; cch < 8; ++cch) {
                 uint32_t o[32];
@@ -596,12 +601,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 // column 32*cch of MMA c = cch/4 holds channel 256c + 128*half + 32*(cch%4)
                 const int ch = 256 * (cch >> 2) + 128 * half + 32 * (cch & 3);
 #pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
+                for (int pc = 0; pc < 4; ++pc) {
                     __syncwarp();   // the previous piece has been read back
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int j = 16 * pc + 4 * c;
-                        st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4),
+                    for (int c = 0; c < 2; ++c) {
+                        const int j = 8 * pc + 4 * c;
+                        st_shared_v4(stg + lane * 32 + ((c ^ ((lane >> 2) & 1)) << 4),
                                      __float_as_uint(__uint_as_float(o[j]) * inv),
                                      __float_as_uint(__uint_as_float(o[j + 1]) * inv),
                                      __float_as_uint(__uint_as_float(o[j + 2]) * inv),
@@ -609,13 +614,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                     __syncwarp();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = rr + 8 * i;                         // staging row = lane r of this warp
+                    for (int i = 0; i < 2; ++i) {
+                        const int r = rr + 16 * i;                        // staging row = lane r of this warp
                         const int grow_r = ROWS_CTA * static_cast<int>(rank) + ((q4 * 32 + r) & 63);
-                        const uint4 v = ld_shared_v4(stg + r * 64 + ((rc ^ ((r >> 1) & 3)) << 4));
+                        const uint4 v = ld_shared_v4(stg + r * 32 + ((rc ^ ((r >> 2) & 1)) << 4));
                         if (grow_r < args.rows)
                             *reinterpret_cast<uint4 *>(args.o_part + (slot * args.rows + grow_r) * DC + ch +
-                                                       16 * pc + 4 * rc) = v;
+                                                       8 * pc + 4 * rc) = v;
                     }
                 }
             }
@@ -659,15 +664,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             float l_run = 0.f;            // this lane's share of the row sum
             bool ok = true;
             for (int64_t t = t_begin; t < t_end; ++t, ++k) {
-                const int s = static_cast<int>(k & 1);
-                if (!wait_bounded<false>(bar(&misc->s_full[s]), (k >> 1) & 1, abort_flag,
+                const int s = static_cast<int>(k & 1);          // P buffer, exchange words
+                const int sb = static_cast<int>(k % NSB);       // score buffer
+                if (!wait_bounded<false>(bar(&misc->s_full[sb]), (k / NSB) & 1, abort_flag,
                                          args.timeout_ns)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
                 uint32_t sr[32];
-                ptx::tmem_ld32(tmem + lane_base + TMEM_S + 32 * s, sr);
+                ptx::tmem_ld32(tmem + lane_base + TMEM_S + 32 * sb, sr);
                 ptx::tmem_wait_ld();
 
                 const int32_t tok0 = static_cast<int32_t>(t) * TOK + half * OWN;
@@ -730,9 +736,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                     ptx::tmem_wait_st();
                 }
-                // P buffer s is free: the value product of tile k-2 was issued
-                // before QK^T of tile k (score-buffer rule) and MMAs retire in
-                // issue order, so it finished before s_full(k) arrived.
+                // P buffer s is free once the value product of tile k - 2 is done
+                if (k >= 2 && !wait_bounded<false>(bar(&misc->pv_done[s]), ((k >> 1) - 1) & 1,
+                                                   abort_flag, args.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t pb = base + OFF_P + s * P_BYTES;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
