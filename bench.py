@@ -2,7 +2,7 @@
 """Benchmark: MLA decode over a paged latent cache on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload long|dsv3|ragged|retrofit|tiny|prefill]
+                    [--workload long|dsv3|ragged|retrofit|tiny|prefill] [--cache bf16|fp8]
 
 A step is one pass of the whole decode path -- absorb-in, split-KV decode, and
 the log-sum-exp combine fused with absorb-out (mla_combine_absorb_out; with
@@ -12,6 +12,11 @@ page_size 64, shuffled page table). Inputs (1.2 GB of latent cache) exceed the
 126 MB L2, so no flush is needed between steps. With N GPUs each rank runs its
 own replica (no collective on the data path; weak scaling) and the time is the
 maximum over ranks. One JSON line is printed by rank 0.
+
+--cache fp8 keeps the latent cache as E4M3 codes with one fp32 scale per token
+(k_R stays bf16) and decodes with mla_decode_splitkv_fp8: 644 instead of 1152
+bytes of HBM traffic per cached token (d_c 512 workloads only; reported under
+its own metric name, not the bf16 headline).
 
 --workload prefill times the decompress branch instead: a step is one prefill
 of batch 8 x 4096 prompt tokens (decompression of K_nope / V, then causal
@@ -35,6 +40,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MLA decode KV-tokens/s per B200 (bf16) + % of HBM/tensor roofline vs CPU oracle"
+FP8_METRIC = ("MLA decode KV-tokens/s per B200 (E4M3 latent cache, bf16 products) + % of HBM/tensor "
+              "roofline vs CPU oracle")
 UNIT = "KV-tokens/s"
 PREFILL_METRIC = "MLA prefill (decompress branch) query tokens/s per B200 (bf16) + % of tensor roofline"
 PREFILL_UNIT = "query-tokens/s"
@@ -45,10 +52,10 @@ EV_EVERY = 8
 L2_FLUSH_BYTES = 3 * 126 * 1024 * 1024
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM bytes per launch of the decode kernel from an ncu capture, keyed by the
-# sha256 of the kernel source it was taken on; reported only while the source
-# is unchanged.
-TRAFFIC = {'4256b19f7d42832f': 1220468992}  # decode_pair_kernel, long workload (B16 L65536)
+# DRAM bytes per launch of the decode kernel from an ncu capture, keyed by
+# (sha256 of the kernel source it was taken on, workload, cache format);
+# reported only while the source is unchanged.
+TRAFFIC = {}
 
 
 def _args():
@@ -60,6 +67,8 @@ def _args():
     ap.add_argument("--workload", default="long")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--cache", choices=["bf16", "fp8"], default="bf16",
+                    help="latent cache format (fp8: E4M3 codes + per-token scales)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="run combine and absorb-out as two calls instead of the fused one")
@@ -302,6 +311,23 @@ def run_reference(a):
     return 0
 
 
+def _quantize_pool(api, d, dims, dev):
+    """The E4M3 cache (codes, scales) of every slot of the bf16 c_KV pool, written by
+    the library's quantiser through an identity page table (k_R rewritten unchanged)."""
+    import torch
+    pool = d["ckv_pool"]
+    pages = pool.shape[0]
+    codes, scales = api.alloc_fp8_cache(pages, pool.shape[2], dev)
+    table = torch.arange(pages, dtype=torch.int32, device=dev)[None]
+    pos = torch.arange(pages * 64, dtype=torch.int32, device=dev)
+    seq = torch.zeros_like(pos)
+    api.append_kv_fp8(pool.view(-1, pool.shape[2]), d["kr_pool"].view(-1, d["kr_pool"].shape[2]),
+                      seq, pos, codes, scales, d["kr_pool"], table, dims, theta=0.0)
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    return codes, scales
+
+
 def cpu_baseline(w, inp, target_s):
     """Oracle (absorbed fp64 path, all host cores) on a bounded sample of rows."""
     import numpy as np
@@ -362,10 +388,15 @@ def main():
     dec = api.Decoder(dims, w.batch, d["block_table"].shape[1], total_tiles, dev)
     stream = torch.cuda.current_stream()
     tokens_per_step = float(lens.sum())
+    fp8 = a.cache == "fp8"
+    if fp8:
+        assert w.d_latent == 512, "the E4M3 decode serves d_c 512 workloads"
+        d["codes"], d["scales"] = _quantize_pool(api, d, dims, dev)
+        del d["ckv_pool"]
     # Model state of one layer: the latent cache and the two absorbed weights. When
     # it fits in L2, the steps walk over several layers' copies (a model's layers
     # each own a cache and weights), so that no step finds its operands in L2.
-    state_keys = ("ckv_pool", "kr_pool", "w_uk", "w_uv")
+    state_keys = (("codes", "scales") if fp8 else ("ckv_pool",)) + ("kr_pool", "w_uk", "w_uv")
     layer_bytes = sum(d[k].numel() * d[k].element_size() for k in state_keys)
     n_layers = max(1, math.ceil(L2_FLUSH_BYTES / layer_bytes))
     layers = [d] + [{k: d[k].clone() for k in state_keys} for _ in range(n_layers - 1)]
@@ -379,8 +410,12 @@ def main():
         api.absorb_q(x["q_c"], x["q_r"], m["w_uk"], dims, out=dec.q)
         if ev is not None:
             ev[0].record(stream)
-        api.decode_splitkv(dec.q, m["ckv_pool"], m["kr_pool"], x["block_table"], x["seq_lens"],
-                           dims, dec.num_parts, workspace=dec.workspace)
+        if fp8:
+            api.decode_splitkv_fp8(dec.q, m["codes"], m["scales"], m["kr_pool"], x["block_table"],
+                                   x["seq_lens"], dims, dec.num_parts, workspace=dec.workspace)
+        else:
+            api.decode_splitkv(dec.q, m["ckv_pool"], m["kr_pool"], x["block_table"], x["seq_lens"],
+                               dims, dec.num_parts, workspace=dec.workspace)
         if ev is not None:
             ev[1].record(stream)
         if a.unfused:
@@ -494,15 +529,16 @@ def main():
 
     hbm, tflops, src = _peaks()
     R = w.n_q * w.heads
-    kv_bytes = tokens_per_step * (w.d_latent + w.d_rope) * 2
+    kv_bytes = tokens_per_step * ((w.d_latent + 4 + 2 * w.d_rope) if fp8 else (w.d_latent + w.d_rope) * 2)
     q_bytes = w.batch * R * (w.d_latent + w.d_rope) * 2
     alg_bytes = kv_bytes + q_bytes
     vis = sum(sum(int(L) - w.n_q + i + 1 for i in range(w.n_q)) for L in lens)
     alg_flops = vis * w.heads * (2 * (w.d_latent + w.d_rope) + 2 * w.d_latent)
     achieved = alg_bytes / (decode_ms / 1e3) / 1e9
-    tr = TRAFFIC.get(_src_hash())
+    tr = TRAFFIC.get((_src_hash(), w.name, a.cache))
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": tr, "kernel": "decode_pair_kernel"
+            "frac": achieved / hbm, "traffic": tr, "kernel": ("decode_pair_kernel<true>" if fp8 else
+                                                              "decode_pair_kernel<false>")
             if w.d_latent == 512 else "decode_single_kernel",
             "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
             "algorithmic_bytes_per_launch": alg_bytes,
@@ -512,12 +548,15 @@ def main():
             "tensor_frac": alg_flops / (decode_ms / 1e3) / 1e12 / tflops}
 
     clocks = sampler.summary(wall0, wall1)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+    line = {"metric": FP8_METRIC if fp8 else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": _workload_desc(w, lens), "batch": w.batch,
                        "seq_len": w.seq_len or list(w.ragged), "heads": w.heads,
                        "kv_tokens_per_step": tokens_per_step, "num_parts": dec.num_parts,
+                       "cache": ("E4M3 c_KV codes + fp32 per-token scales, bf16 k_R (644 B/token)"
+                                 if fp8 else "bf16 c_KV and k_R (1152 B/token)"),
                        "l2": ("inputs larger than L2 (latent cache %.2f GB), no flush" % (kv_bytes / 1e9)
                               if n_layers == 1 else
                               "inputs larger than L2: steps cycle over %d layers' copies of the "
@@ -525,7 +564,8 @@ def main():
                               % (n_layers, n_layers * layer_bytes / 1e9)),
                        "layers": n_layers,
                        "parallelism": "replicas" if world > 1 else "single",
-                       "step_calls": ["mla_absorb_q", "mla_decode_splitkv"] +
+                       "step_calls": ["mla_absorb_q",
+                                      "mla_decode_splitkv_fp8" if fp8 else "mla_decode_splitkv"] +
                                      (["mla_combine", "mla_absorb_out"] if a.unfused
                                       else ["mla_combine_absorb_out"])},
             "roofline": roof,

@@ -431,6 +431,27 @@ mla_status mla_decompress_kv_fp8(const mla_dims *dims, const mla_pool *ckv8, con
                                  const void *w_uk, const void *w_uv, void *workspace,
                                  size_t workspace_bytes, void *stream);
 
+/* mla_decode_splitkv reading the E4M3 cache (the quantised latent-cache gather
+ * that the "MLA operator design" page places on the decode side, introduction
+ * and §5): c_KV comes from the codes pool and its per-token scales, k_R from
+ * the bf16 pool. Each c_KV element is dequantised as above before it enters
+ * either product, so the result is mla_decode_splitkv's on the dequantised
+ * bf16 cache: HBM traffic per cached token is 512 code bytes + a 4-byte scale
+ * + 128 bytes of k_R (644) instead of 1152. Elements past a sequence's end in
+ * its last page never reach a product, whatever their codes or scale.
+ * d_latent 512 / d_rope 64 only (else MLA_ERR_UNSUPPORTED); the workspace,
+ * partition plan and the other arguments are those of mla_decode_splitkv, and
+ * mla_combine reads the workspace unchanged.
+ * ckv8    codes pool [pages, 64, >= 512] uint8 (strides in bytes, base and
+ *         strides multiples of 16)
+ * scales  [num_pages, 64] fp32, dense, 16-byte aligned base
+ */
+mla_status mla_decode_splitkv_fp8(const mla_dims *dims, const void *q, const mla_pool *ckv8,
+                                  const float *scales, const mla_pool *kr, int32_t num_pages,
+                                  const int32_t *block_table, int32_t max_pages_per_seq,
+                                  const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ EXPORTS = ("mla_absorb_q", "mla_decode_num_parts", "mla_decode_workspace_bytes",
            "mla_absorb_q_rope", "mla_prefill_workspace_bytes", "mla_decompress_kv",
            "mla_prefill_attention", "mla_prefill", "mla_append_kv",
            "mla_append_kv_fp8", "mla_gather_dequant_fp8", "mla_decompress_kv_fp8",
-           "mla_default_num_splits", "mla_decode_workspace_size")
+           "mla_default_num_splits", "mla_decode_workspace_size", "mla_decode_splitkv_fp8")
 
 
 class MLADims(ctypes.Structure):
@@ -75,6 +75,7 @@ def _load():
         "mla_decompress_kv_fp8": (i32, [D, PL, P, i32, P, i32, P, i32, P, P, P, sz, P]),
         "mla_default_num_splits": (i32, [D, i32, i32, i32]),
         "mla_decode_workspace_size": (sz, [D, i32, i32]),
+        "mla_decode_splitkv_fp8": (i32, [D, P, PL, P, PL, i32, P, i32, P, i32, i32, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

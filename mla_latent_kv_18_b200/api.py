@@ -123,6 +123,24 @@ def decode_splitkv(q, ckv_pool, kr_pool, block_table, seq_lens, dims, num_parts,
     return workspace
 
 
+def decode_splitkv_fp8(q, ckv8_pool, scales, kr_pool, block_table, seq_lens, dims, num_parts,
+                       workspace=None, stream=None):
+    """decode_splitkv reading the E4M3 cache (codes [pages, 64, 512] uint8, scales
+    [pages, 64] fp32, k_R bf16); combine() reads the workspace as usual."""
+    B = block_table.shape[0]
+    if workspace is None:
+        workspace = alloc_workspace(dims, B, num_parts, q.device)
+    assert scales.dtype == torch.float32 and scales.is_contiguous()
+    _b.check(_b.lib.mla_decode_splitkv_fp8(ctypes.byref(dims), _ptr(q),
+                                           ctypes.byref(_pool8(ckv8_pool)), _ptr(scales),
+                                           ctypes.byref(_pool(kr_pool)), ckv8_pool.shape[0],
+                                           _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
+                                           B, num_parts, _ptr(workspace), workspace.numel(),
+                                           _stream(stream)),
+             "mla_decode_splitkv_fp8")
+    return workspace
+
+
 def combine(workspace, seq_lens, max_pages, dims, num_parts, o_lat=None, lse_out=None,
             with_lse=True, stream=None):
     B = seq_lens.shape[0]

@@ -3,6 +3,8 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "ptx.cuh"
 
@@ -72,6 +74,57 @@ __device__ __forceinline__ bool wait_word(const uint32_t *slot, uint32_t tag,
             }
         }
     }
+}
+
+// Multiply written in PTX so that no flush-to-zero applies whatever the
+// compile flags (subnormal products stay exact, as in the definition).
+__device__ __forceinline__ float mul_rn_noftz(float a, float b) {
+    float d;
+    asm("mul.rn.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// E4M3 dequantisation: bf16_rn( fp32_rn( value(code) * scale ) ). value(code)
+// is exact in fp16 and fp32, so only the product and the final narrowing round.
+// Two codes (the low byte is the first) to a bf16 pair (the first in the low half).
+__device__ __forceinline__ uint32_t dequant2_e4m3(uint32_t two_codes, float scale) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu),
+                                                     __NV_E4M3);
+    const float2 f = __half22float2(__half2(h));
+    const __nv_bfloat162 v = __floats2bfloat162_rn(mul_rn_noftz(f.x, scale), mul_rn_noftz(f.y, scale));
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// 8 codes (two 32-bit words) to 8 bf16.
+__device__ __forceinline__ uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float scale) {
+    return make_uint4(dequant2_e4m3(w0, scale), dequant2_e4m3(w0 >> 16, scale), dequant2_e4m3(w1, scale),
+                      dequant2_e4m3(w1 >> 16, scale));
+}
+
+// 4 codes (a 32-bit word, first code in the low byte) to 4 bf16 as two words:
+// codes -> f16 pairs (exact) -> fp32 (exact) -> product (rounded once) -> bf16,
+// the same arithmetic as dequant2_e4m3 in fewer instructions.
+__device__ __forceinline__ uint2 dequant4_e4m3(uint32_t w, float scale) {
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(h01), "=r"(h23)
+        : "r"(w));
+    float f[4];
+    asm("{\n\t.reg .b16 a, b, c, d;\n\tmov.b32 {a, b}, %4;\n\tmov.b32 {c, d}, %5;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\tcvt.f32.f16 %2, c;\n\tcvt.f32.f16 %3, d;\n\t}"
+        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
+        : "r"(h01), "r"(h23));
+    // products two at a time (mul.rn.f32x2, no flush-to-zero)
+    float p[4];
+    asm("{\n\t.reg .b64 A, B, S, D, E;\n\tmov.b64 A, {%4, %5};\n\tmov.b64 B, {%6, %7};\n\t"
+        "mov.b64 S, {%8, %8};\n\tmul.rn.f32x2 D, A, S;\n\tmul.rn.f32x2 E, B, S;\n\t"
+        "mov.b64 {%0, %1}, D;\n\tmov.b64 {%2, %3}, E;\n\t}"
+        : "=f"(p[0]), "=f"(p[1]), "=f"(p[2]), "=f"(p[3])
+        : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(scale));
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(p[0], p[1]);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(p[2], p[3]);
+    return make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
 }
 
 // ---------------------------------------------------------------------------

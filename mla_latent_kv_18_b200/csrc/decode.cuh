@@ -40,6 +40,7 @@ struct DecodeArgs {
     const __nv_bfloat16 *q;      // [B, R, D]
     const int32_t *block_table;  // [B, max_pages]
     const int32_t *seq_lens;     // [B]
+    const float *kv_scales;      // E4M3 cache: per-token scales [pages, 64] (else unused)
     float *o_part;               // [slots, R, d_c]
     float *lse_part;             // [slots, R]
     int64_t timeout_ns;
@@ -57,6 +58,8 @@ struct DecodeArgs {
 constexpr int kDecodeThreads = 192;          // single kernel: 6 warps
 constexpr int kPairThreads = 352;            // pair kernel: 11 warps (6 = P.V-slot producer, 7..10 segment warps)
 constexpr int kSegWarp0 = 7;                 // pair kernel: first of the four segment warps
+constexpr int kPairThreadsFp8 = 480;         // E4M3 pair kernel: + 4 dequantising warps (11..14)
+constexpr int kDqWarp0 = 11;
 constexpr int kSoftmaxWarp0 = 2;             // warps 2..5
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when max grows > 2^8
 
@@ -180,6 +183,11 @@ constexpr uint32_t TMEM_S = 256;               // three 32-column score buffers
 constexpr uint32_t TMEM_Q = TMEM_S + NSB * 32; // Q blocks 0..4: 32 columns each (two bf16 per column)
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, 256, 0, 1);
+// E4M3 cache: a slot's c_KV codes land in bytes [CODE_OFF, CODE_OFF + CODE_BYTES)
+// of the slot and are widened in place to the bf16 operand above.
+constexpr uint32_t CODE_OFF = 16384;
+constexpr uint32_t CODE_BYTES = 16384;         // QK^T: 32 tokens x 512; P.V: 64 tokens x 256
+constexpr uint32_t SC_BYTES = 4 * 32 * 4;      // four copies of 32 tokens' scales per slot
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(TMEM_Q + QT * 32 <= TMEM_COLS, "tensor memory budget");
 static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 0 &&
@@ -203,13 +211,144 @@ struct Misc {
     uint64_t q_free;                  // pair kernel: the last QK^T of a segment is done (Q may be replaced)
     uint64_t seg_done;                // pair kernel: a segment's row sums and maxima are published
     float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
+    uint64_t code_qk[pair::QK_STAGES], code_pv[pair::PV_STAGES];   // E4M3 pair kernel: codes landed
 };
 static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+// Tile-by-tile walk over a partition's segments.
+struct TileCursor {
+    SegmentWalker w;
+    bool have;
+    int64_t t;   // tile index within sequence w.seg_b
+    __device__ void start() {
+        have = w.next();
+        t = have ? w.t_begin : 0;
+    }
+    __device__ void advance() {
+        if (++t >= w.t_end) {
+            have = w.next();
+            if (have) t = w.t_begin;
+        }
+    }
+};
+
+// E4M3 pair kernel: one warp widens its share of a ring slot's codes in place.
+// The codes sit at slot + CODE_OFF as NBOX boxes of [rows x 128 codes] (box v:
+// 128 consecutive channels of the slot's channel range, rows = blk / 128); the
+// bf16 operand is block j = 2v + e ([rows x 64 channels], 128-byte swizzled) at
+// slot + j * blk. The warp owns 8 NPAIR slot rows from wrow0 on; lane
+// (c = lane & 7, q = lane >> 3) converts 16-code chunk c of rows
+// row(pr, h) = wrow0 + 2 (q + 4 pr) + ((c / 4) ^ h) & 1 of every box, for its
+// NPAIR row pairs pr. A quarter-warp's two rows alternate with c, so its reads
+// cover 128 contiguous bytes and its stores fall in distinct banks. The units
+// (box, pr) go in order, two per step: a step's codes are read by every lane
+// before the warp syncs and any lane writes the step's outputs. An output row
+// overlaps only codes of the same row, of this box or an earlier one, so every
+// code is read before it is overwritten; the next step's codes (never written
+// by this step) are loaded before this step's stores, which hides the load
+// latency. Rows at or past rlim (tokens past the sequence end) are written as
+// zeros. The loop stays rolled: one step of straight-line code.
+template <int NBOX, int NPAIR>
+__device__ __forceinline__ void dequant_slot(uint32_t slot, uint32_t blk, int wrow0, int lane, int32_t rlim,
+                                             const float (&sc)[2 * NPAIR]) {
+    constexpr int NST = NBOX * NPAIR / 2;   // steps of two units
+    static_assert(NPAIR <= 2, "a step's scales are fixed");
+    const int c = lane & 7, q = lane >> 3;
+    const uint32_t codes = slot + pair::CODE_OFF + c * 16;
+    auto row = [&](int pr, int h) { return wrow0 + 2 * (q + 4 * pr) + (((c >> 2) ^ h) & 1); };
+    // row(pr, h) mod 8 does not depend on pr, so neither do the swizzled chunk
+    // offsets of the two 16-byte outputs: (2 (c mod 4) + x) ^ (row mod 8), x = 0, 1
+    uint32_t xo[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int x = 0; x < 2; ++x) xo[h][x] = static_cast<uint32_t>(((2 * (c & 3) + x) ^ (row(0, h) & 7)) << 4);
+    // unit un: box un / NPAIR, pair un % NPAIR (compile-time within a step but for the box)
+    auto load = [&](int st, uint4 (&v)[4]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int un = 2 * st + (u >> 1);
+            v[u] = ld_shared_v4(codes + (un / NPAIR) * blk + row(un % NPAIR, u & 1) * 128);
+        }
+    };
+    uint4 v[4];
+    load(0, v);
+#pragma unroll 1
+    for (int st = 0; st < NST; ++st) {
+        __syncwarp();   // every lane has read this step's codes
+        uint4 o[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            // scale of row(pr, h): entry 2 pr + h; within a step pr = (2 st + u / 2) % NPAIR
+            // is u / 2 for NPAIR 2 and 0 for NPAIR 1
+            const float s = sc[(NPAIR == 2 ? 2 * (u >> 1) : 0) + (u & 1)];
+            const uint2 d0 = dequant4_e4m3(v[u].x, s);
+            const uint2 d1 = dequant4_e4m3(v[u].y, s);
+            const uint2 d2 = dequant4_e4m3(v[u].z, s);
+            const uint2 d3 = dequant4_e4m3(v[u].w, s);
+            o[2 * u] = make_uint4(d0.x, d0.y, d1.x, d1.y);
+            o[2 * u + 1] = make_uint4(d2.x, d2.y, d3.x, d3.y);
+        }
+        uint4 nv[4];
+        if (st + 1 < NST) load(st + 1, nv);   // the next step's codes: rows or boxes this step does not write
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int un = 2 * st + (u >> 1);
+            const int r = row(un % NPAIR, u & 1);
+            uint4 lo = o[2 * u], hi = o[2 * u + 1];
+            if (r >= rlim) lo = hi = make_uint4(0u, 0u, 0u, 0u);
+            // sw128(r, chunk) = r * 128 + xo
+            const uint32_t rb = slot + (2 * (un / NPAIR) + (c >> 2)) * blk + static_cast<uint32_t>(r) * 128u;
+            st_shared_v4(rb + xo[u & 1][0], lo.x, lo.y, lo.z, lo.w);
+            st_shared_v4(rb + xo[u & 1][1], hi.x, hi.y, hi.z, hi.w);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = nv[u];
+    }
+}
+
+// E4M3 pair kernel: one dequantising warp's share of one slot: wait until the
+// slot's codes and scales have landed, widen them, report the slot full on the
+// leader's barrier. The scales (32 consecutive tokens, from slot row sc_row0
+// on) arrive by TMA in the warp's own last row of block NBOX - 1, which the
+// warp itself overwrites in its first step, after reading them.
+template <int NBOX, int NPAIR>
+__device__ __forceinline__ bool dequant_tile(const TileCursor &cur, int64_t k, const DecodeArgs &args,
+                                             uint32_t ring, uint32_t stage, uint32_t blk, int nst,
+                                             uint64_t *codeb, uint64_t *fullb, int wrow0, int sc_row0,
+                                             int tok_off, uint32_t rank, int lane,
+                                             volatile int32_t *abort_flag) {
+    const int c = lane & 7, q = lane >> 3;
+    const int s = static_cast<int>(k % nst);
+    if (!wait_bounded<false>(ptx::smem_u32(&codeb[s]), (k / nst) & 1, abort_flag, args.timeout_ns))
+        return false;
+    const uint32_t slot = ring + s * stage;
+    const uint32_t sc_off = (NBOX - 1) * blk + (wrow0 + 8 * NPAIR - 1) * 128;
+    float sc[2 * NPAIR];
+#pragma unroll
+    for (int i = 0; i < 2 * NPAIR; ++i) {
+        const int r = wrow0 + 2 * (q + 4 * (i >> 1)) + (((c >> 2) ^ i) & 1);
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc[i]) : "r"(slot + sc_off + 4 * (r - sc_row0)) : "memory");
+    }
+    __syncwarp();   // the scale row is overwritten below
+    const int32_t rlim = cur.w.L - static_cast<int32_t>(cur.t) * pair::TOK - tok_off;
+    dequant_slot<NBOX, NPAIR>(slot, blk, wrow0, lane, rlim, sc);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        const uint32_t fb = ptx::smem_u32(&fullb[s]);
+        if (rank == 0) ptx::mbar_arrive(fb);
+        else ptx::mbar_arrive_cluster(ptx::mapa(fb, 0));
+    }
+    return true;
+}
+
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsFp8 : kPairThreads, 1)
     decode_pair_kernel(const __grid_constant__ CUtensorMap map_ckv32,
                        const __grid_constant__ CUtensorMap map_ckv64,
-                       const __grid_constant__ CUtensorMap map_kr32, const DecodeArgs args) {
+                       const __grid_constant__ CUtensorMap map_kr32,
+                       const __grid_constant__ CUtensorMap map_sc, const DecodeArgs args) {
     using namespace pair;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = ptx::smem_u32(smem_raw);
@@ -233,14 +372,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
+        // E4M3: a slot is full once the eight dequantising warps of the pair
+        // have widened it (and, for QK^T, the leader's k_R copies have landed)
         for (int i = 0; i < QK_STAGES; ++i) {
-            ptx::mbar_init(bar(&misc->qk_full[i]), 1);
+            ptx::mbar_init(bar(&misc->qk_full[i]), kFp8 ? 9 : 1);
             ptx::mbar_init(bar(&misc->qk_empty[i]), 1);
+            if (kFp8) ptx::mbar_init(bar(&misc->code_qk[i]), 1);
         }
         for (int i = 0; i < PV_STAGES; ++i) {
-            ptx::mbar_init(bar(&misc->pv_full[i]), 1);
+            ptx::mbar_init(bar(&misc->pv_full[i]), kFp8 ? 8 : 1);
             ptx::mbar_init(bar(&misc->pv_empty[i]), 1);
             ptx::mbar_init(bar(&misc->pv_landed[i]), 1);
+            if (kFp8) ptx::mbar_init(bar(&misc->code_pv[i]), 1);
         }
         for (int i = 0; i < NSB; ++i) ptx::mbar_init(bar(&misc->s_full[i]), 1);
         for (int i = 0; i < 2; ++i) {
@@ -279,6 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ptx::prefetch_tensormap(&map_ckv32);
             ptx::prefetch_tensormap(&map_ckv64);
             ptx::prefetch_tensormap(&map_kr32);
+            if (kFp8) ptx::prefetch_tensormap(&map_sc);
         }
     }
     ptx::tc_fence_before();
@@ -310,13 +454,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // ------------------------------------------------------ TMA producers
         // warp 0 fills the QK^T ring (own 32 tokens x 9 channel blocks), warp 6
         // the P.V ring (64 tokens x this SM's 4 channel blocks). Completion of
-        // both CTAs' copies is counted on the leader's barriers.
+        // both CTAs' copies is counted on the leader's barriers. E4M3: the c_KV
+        // codes of a slot land on this CTA's own barrier (code_qk / code_pv) for
+        // the dequantising warps; k_R (bf16) still lands on the leader's.
         const bool qk = (warp == 0);
         if (ptx::elect_one()) {
             uint64_t *fullb = qk ? misc->qk_full : misc->pv_full;
             uint64_t *emptyb = qk ? misc->qk_empty : misc->pv_empty;
+            uint64_t *codeb = qk ? misc->code_qk : misc->code_pv;
             const int nst = qk ? QK_STAGES : PV_STAGES;
-            const uint32_t tx = 2 * (qk ? STAGE_QK : STAGE_PV);
+            const uint32_t tx = kFp8 ? 2 * (OWN * 128) : 2 * (qk ? STAGE_QK : STAGE_PV);
             int64_t k = 0;
             bool bad_page = false;
             while (!*abort_flag && walk.next()) {
@@ -330,6 +477,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                                   args.timeout_ns))
                         break;
                     const uint32_t fb = (rank == 0) ? bar(&fullb[s]) : leader_bar(&fullb[s]);
+                    if constexpr (kFp8) {
+                        // codes, then 32 tokens' scales for each dequantising warp
+                        // into that warp's last row of block 3 (QK^T) or 1 (P.V)
+                        const uint32_t cb = bar(&codeb[s]);
+                        ptx::mbar_arrive_expect_tx(cb, CODE_BYTES + SC_BYTES);
+                        if (qk) {
+                            const uint32_t st = base + OFF_QK + s * STAGE_QK;
+                            for (int i = 0; i < 4; ++i)   // [32 own tokens x 128 codes] boxes
+                                ptx::tma_load_3d(st + CODE_OFF + i * (OWN * 128), &map_ckv32, cb, 128 * i,
+                                                 OWN * rank, page);
+                            for (int w = 0; w < 4; ++w)   // dequantising warp w: row 8w + 7 of block 3
+                                ptx::tma_load_2d(st + 3 * (OWN * 128) + (8 * w + 7) * 128, &map_sc, cb,
+                                                 OWN * rank, page);
+                            if (rank == 0) ptx::mbar_arrive_expect_tx(fb, tx);
+                            ptx::tma_load_3d_pair(st + 8 * (OWN * 128), &map_kr32, fb, 0, OWN * rank, page);
+                        } else {
+                            const uint32_t st = base + OFF_PV + s * STAGE_PV;
+                            for (int v = 0; v < 2; ++v)   // this SM's channels 256v + 128 rank + [0, 128)
+                                for (int h = 0; h < 2; ++h)
+                                    ptx::tma_load_3d(st + CODE_OFF + v * (TOK * 128) + h * (OWN * 128),
+                                                     &map_ckv32, cb, 256 * v + 128 * static_cast<int>(rank),
+                                                     OWN * h, page);
+                            for (int w = 0; w < 4; ++w)   // dequantising warp w: row 16w + 15 of block 1
+                                ptx::tma_load_2d(st + 1 * (TOK * 128) + (16 * w + 15) * 128, &map_sc, cb,
+                                                 OWN * (w >> 1), page);
+                        }
+                        continue;
+                    }
                     if (rank == 0) ptx::mbar_arrive_expect_tx(fb, tx);
                     if (qk) {
                         const uint32_t st = base + OFF_QK + s * STAGE_QK;
@@ -349,7 +524,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
             if (bad_page) record_error(kErrDeviceBounds);
             // drain: the leader waits until every issued slot has landed
-            if (rank == 0) {
+            // (E4M3: each CTA waits for its own code copies)
+            if (kFp8) {
+                for (int64_t kk = (k >= nst ? k - nst : 0); kk < k; ++kk)
+                    wait_bounded<false>(bar(&codeb[kk % nst]), (kk / nst) & 1, abort_flag, args.timeout_ns);
+            } else if (rank == 0) {
                 for (int64_t kk = (k >= nst ? k - nst : 0); kk < k; ++kk)
                     wait_bounded(bar(&fullb[kk % nst]), (kk / nst) & 1, abort_flag, args.timeout_ns);
             }
@@ -471,6 +650,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             // every MMA issued so far has finished before tensor memory is freed
             ptx::mma_commit_pair(bar(&misc->drain), 0x1);
             wait_bounded<false>(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
+        }
+    } else if (kFp8 && warp >= kDqWarp0) {
+        // ------------------------------------------------------ dequantising warps
+        if constexpr (kFp8) {
+            const int dq = warp - kDqWarp0;
+            // every warp takes 8 of a QK^T slot's 32 rows and 16 of a P.V slot's
+            // 64, converting QK^T one tile ahead of P.V (the MMAs consume them in
+            // that order); the scale copies hold the CTA's 32 QK^T tokens and
+            // P.V tokens 32 (dq / 2) + [0, 32)
+            TileCursor cq, cp;
+            cq.w = walk;
+            cq.start();
+            cp = cq;
+            int64_t kq = 0, kp = 0;
+            bool ok = true;
+            auto qk_tile = [&]() {
+                ok = dequant_tile<4, 1>(cq, kq, args, base + OFF_QK, STAGE_QK, OWN * 128, QK_STAGES, misc->code_qk,
+                                        misc->qk_full, 8 * dq, 0, OWN * static_cast<int>(rank), rank, lane,
+                                        abort_flag);
+                cq.advance();
+                ++kq;
+            };
+            if (cq.have) qk_tile();
+            while (ok && cp.have && !*abort_flag) {
+                if (cq.have) qk_tile();
+                if (!ok) break;
+                ok = dequant_tile<2, 2>(cp, kp, args, base + OFF_PV, STAGE_PV, TOK * 128, PV_STAGES, misc->code_pv,
+                                        misc->pv_full, 16 * dq, 32 * (dq >> 1), 0, rank, lane, abort_flag);
+                cp.advance();
+                ++kp;
+            }
         }
     } else if (warp >= kSegWarp0) {
         // ------------------------------------------------------ segment warps
@@ -756,7 +966,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 // slot). Their P is 0, but 0 * NaN = NaN in the value product, so
                 // they are cleared in this CTA's P.V slot once it has landed.
                 const int32_t valid = L - static_cast<int32_t>(t) * TOK;
-                if (valid < TOK) {
+                if (!kFp8 && valid < TOK) {   // (E4M3: the dequantising warps wrote zeros there)
                     const int ps = static_cast<int>(k % PV_STAGES);
                     if (!wait_bounded(bar(&misc->pv_landed[ps]), (k / PV_STAGES) & 1, abort_flag,
                                       args.timeout_ns)) {

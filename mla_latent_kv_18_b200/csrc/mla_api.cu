@@ -77,7 +77,9 @@ mla_status device_ready() {
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { st.status = MLA_ERR_CUDA; return; }
         if (prop.major != 10 || prop.minor != 0) { st.status = MLA_ERR_UNSUPPORTED; return; }
-        if (cudaFuncSetAttribute(mla::decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(mla::decode_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::pair::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::pair::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_single_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -109,7 +111,9 @@ mla_status device_ready() {
                 cudaSuccess ||
             cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  carve) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::decode_pair_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+            cudaFuncSetAttribute(mla::decode_pair_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carve) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_pair_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  carve) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_single_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  carve) != cudaSuccess) {
@@ -226,6 +230,38 @@ mla_status launch_proj(const void *x, const void *w, void *out, const void *rope
     dim3 grid(H, (n_cols + 127) / 128, (T + NT - 1) / NT);
     return launch_pdl(mla::proj_tc_kernel, grid, dim3(128), mla::proj_smem_bytes(NT, a.stages), s, mw, mx,
                       a);
+}
+
+// 3-D uint8 map over an E4M3 code pool: dims (channels, 64 tokens, pages),
+// unswizzled boxes of [box_tok tokens x box_ch codes].
+mla_status code_pool_map(CUtensorMap *m, const mla_pool *pool, int32_t channels, int32_t num_pages,
+                         uint32_t box_ch, uint32_t box_tok) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(channels), 64,
+                                static_cast<cuuint64_t>(num_pages)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pool->token_stride),
+                                   static_cast<cuuint64_t>(pool->page_stride)};
+    const cuuint32_t box[3] = {box_ch, box_tok, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(pool->base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
+}
+
+// 2-D fp32 map over the per-token scales [pages, 64]: boxes of box_tok tokens of one page.
+mla_status scale_map(CUtensorMap *m, const float *scales, int32_t num_pages, uint32_t box_tok) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(num_pages)};
+    const cuuint64_t strides[1] = {64 * sizeof(float)};
+    const cuuint32_t box[2] = {box_tok, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(scales), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
 }
 
 mla_status check_pool(const mla_pool *p, int32_t channels) {
@@ -368,31 +404,21 @@ mla_status mla_absorb_out(const mla_dims *dims, const void *o_lat, const void *w
                        dims->d_v, dims->d_v, 0, static_cast<cudaStream_t>(stream));
 }
 
-mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_pool *ckv,
-                              const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
-                              int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
-                              int32_t num_parts, void *workspace, size_t workspace_bytes,
-                              void *stream) {
-    mla_status st = check_dims(dims, true);
-    if (st != MLA_OK) return st;
-    if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0 || num_pages <= 0)
-        return MLA_ERR_INVALID_ARG;
-    if (batch == 0) return MLA_OK;
-    if (!q || !block_table || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
-        !aligned(workspace, 256))
-        return MLA_ERR_INVALID_ARG;
-    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
-    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
-    if (workspace_bytes < mla_decode_workspace_bytes(dims, batch, num_parts)) return MLA_ERR_INVALID_ARG;
-    if ((st = device_ready()) != MLA_OK) return st;
+}  // extern "C"
 
+namespace {
+// The split-KV arguments common to both cache formats (validated by the caller).
+mla::DecodeArgs decode_args(const mla_dims *dims, const void *q, int32_t num_pages,
+                            const int32_t *block_table, int32_t max_pages_per_seq,
+                            const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                            void *workspace) {
     const int64_t R = static_cast<int64_t>(dims->n_q) * dims->num_heads;
     const int64_t slots = static_cast<int64_t>(batch) + num_parts;
     mla::DecodeArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.block_table = block_table;
     a.seq_lens = seq_lens;
+    a.kv_scales = nullptr;
     a.o_part = static_cast<float *>(workspace);
     a.lse_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                            round_up(slots * R * dims->d_latent * 4, 256));
@@ -406,6 +432,44 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
     a.rows = static_cast<int32_t>(R);
     a.scale = scale_of(dims);
     a.scale_log2 = a.scale * 1.4426950408889634f;
+    return a;
+}
+
+mla_status check_decode_common(const mla_dims *dims, const void *q, int32_t num_pages,
+                               const int32_t *block_table, int32_t max_pages_per_seq,
+                               const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                               void *workspace, size_t workspace_bytes) {
+    if (batch < 0 || num_parts <= 0 || max_pages_per_seq <= 0 || num_pages <= 0)
+        return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    if (!q || !block_table || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+        !aligned(workspace, 256))
+        return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_decode_workspace_bytes(dims, batch, num_parts)) return MLA_ERR_INVALID_ARG;
+    return MLA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_pool *ckv,
+                              const mla_pool *kr, int32_t num_pages, const int32_t *block_table,
+                              int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                              int32_t num_parts, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if ((st = check_decode_common(dims, q, num_pages, block_table, max_pages_per_seq, seq_lens, batch,
+                                  num_parts, workspace, workspace_bytes)) != MLA_OK)
+        return st;
+    if (batch == 0) return MLA_OK;
+    if ((st = check_pool(ckv, dims->d_latent)) != MLA_OK) return st;
+    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    if ((st = device_ready()) != MLA_OK) return st;
+
+    const mla::DecodeArgs a = decode_args(dims, q, num_pages, block_table, max_pages_per_seq, seq_lens,
+                                          batch, num_parts, workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     if (variant_of(dims) == Variant::Pair512) {
@@ -419,8 +483,8 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
         if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
             return st;
-        return launch_pdl(mla::decode_pair_kernel, dim3(2 * num_parts), dim3(mla::kPairThreads),
-                          mla::pair::SMEM_BYTES, s, m32, m64, mkr, a);
+        return launch_pdl(mla::decode_pair_kernel<false>, dim3(2 * num_parts), dim3(mla::kPairThreads),
+                          mla::pair::SMEM_BYTES, s, m32, m64, mkr, mkr /* no scales */, a);
     } else {
         CUtensorMap mc, mkr;
         if ((st = pool_map(&mc, ckv, 64, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
@@ -430,6 +494,38 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
         return launch_pdl(mla::decode_single_kernel, dim3(num_parts), dim3(mla::kDecodeThreads),
                           mla::single::SMEM_BYTES, s, mc, mkr, a);
     }
+}
+
+mla_status mla_decode_splitkv_fp8(const mla_dims *dims, const void *q, const mla_pool *ckv8,
+                                  const float *scales, const mla_pool *kr, int32_t num_pages,
+                                  const int32_t *block_table, int32_t max_pages_per_seq,
+                                  const int32_t *seq_lens, int32_t batch, int32_t num_parts,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    mla_status st = check_dims(dims, true);
+    if (st != MLA_OK) return st;
+    if (variant_of(dims) != Variant::Pair512) return MLA_ERR_UNSUPPORTED;
+    if ((st = check_decode_common(dims, q, num_pages, block_table, max_pages_per_seq, seq_lens, batch,
+                                  num_parts, workspace, workspace_bytes)) != MLA_OK)
+        return st;
+    if (batch == 0) return MLA_OK;
+    if (!ckv8 || !ckv8->base || !aligned(ckv8->base, 16) || ckv8->token_stride < dims->d_latent ||
+        ckv8->page_stride < 64 * ckv8->token_stride || (ckv8->token_stride % 16) ||
+        (ckv8->page_stride % 16))
+        return MLA_ERR_INVALID_ARG;
+    if (!scales || !aligned(scales, 16)) return MLA_ERR_INVALID_ARG;
+    if ((st = check_pool(kr, dims->d_rope)) != MLA_OK) return st;
+    if ((st = device_ready()) != MLA_OK) return st;
+
+    mla::DecodeArgs a = decode_args(dims, q, num_pages, block_table, max_pages_per_seq, seq_lens, batch,
+                                    num_parts, workspace);
+    a.kv_scales = scales;
+    CUtensorMap mc, mkr, msc;
+    if ((st = code_pool_map(&mc, ckv8, 512, num_pages, 128, mla::pair::OWN)) != MLA_OK) return st;
+    if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+        return st;
+    if ((st = scale_map(&msc, scales, num_pages, 32)) != MLA_OK) return st;
+    return launch_pdl(mla::decode_pair_kernel<true>, dim3(2 * num_parts), dim3(mla::kPairThreadsFp8),
+                      mla::pair::SMEM_BYTES, static_cast<cudaStream_t>(stream), mc, mc, mkr, msc, a);
 }
 
 mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t workspace_bytes,

@@ -150,6 +150,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// 2-D tiled load global -> shared::cluster, completion counted on `bar`
+// (a barrier of this CTA).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
 // Same, for a CTA pair: the data lands in this CTA's shared memory while the
 // completion is counted on `bar`, which may be the barrier of the pair's
 // leader CTA (a shared::cluster address obtained with mapa). No multicast.

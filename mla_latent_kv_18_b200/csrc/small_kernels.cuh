@@ -905,24 +905,6 @@ struct GatherFp8Args {
     int32_t width, num_pages, max_pages, batch, max_len;
 };
 
-// 8 E4M3 codes (two 32-bit words, first code in the low byte) to 8 bf16:
-// bf16_rn( fp32_rn( value(code) * scale ) ); value(code) is exact in fp32.
-__device__ __forceinline__ uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float scale) {
-    uint32_t out[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t w = q < 2 ? w0 : w1;
-        const int sh = (q & 1) * 16;
-        __nv_fp8_e4m3 lo, hi;
-        lo.__x = static_cast<__nv_fp8_storage_t>((w >> sh) & 0xFFu);
-        hi.__x = static_cast<__nv_fp8_storage_t>((w >> (sh + 8)) & 0xFFu);
-        const __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(static_cast<float>(lo), scale),
-                                                      __fmul_rn(static_cast<float>(hi), scale));
-        out[q] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-    return make_uint4(out[0], out[1], out[2], out[3]);
-}
-
 __global__ void __launch_bounds__(256) gather_dequant_fp8_kernel(const GatherFp8Args a) {
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);

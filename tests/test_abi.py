@@ -263,6 +263,37 @@ def test_cache_write_and_fp8_calls_validate_without_launch(b):
                                      fake, ws, null) == 1
 
 
+
+def test_fp8_decode_validates_without_launch(b):
+    lib = b.lib
+    by = ctypes.byref
+    d = _dims(b)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x1000)
+    kpool = b.MLAPool(0x1000, 64 * 64, 64)
+    c8 = b.MLAPool(0x1000, 64 * 512, 512)
+    P = 4
+    ws = lib.mla_decode_workspace_bytes(by(d), 2, P)
+
+    def call(dims=d, q=fake, codes=c8, scales=fake, kr=kpool, batch=2, parts=P, wsb=ws,
+             workspace=fake):
+        return lib.mla_decode_splitkv_fp8(by(dims), q, by(codes), scales, by(kr), 8, fake, 4, fake,
+                                          batch, parts, workspace, wsb, null)
+
+    # the 64-wide latent variant has no E4M3 decode
+    small = _dims(b, num_heads=32, n_q=2, d_nope=120, d_latent=64, d_rope=8)
+    assert call(dims=small, wsb=lib.mla_decode_workspace_bytes(by(small), 2, P)) == 2
+    assert call(batch=0) == 0                                           # no-op
+    assert call(scales=null) == 1                                       # scales required
+    assert call(scales=ctypes.c_void_p(0x1004)) == 1                    # 16-byte aligned (TMA)
+    assert call(codes=b.MLAPool(0x1008, 64 * 512, 512)) == 1            # 16-byte base
+    assert call(codes=b.MLAPool(0x1000, 64 * 520, 520)) == 1            # 16-byte strides
+    assert call(codes=b.MLAPool(0x1000, 64 * 256, 256)) == 1            # token stride >= 512
+    assert call(codes=b.MLAPool(0x1000, 32 * 512, 512)) == 1            # page holds 64 tokens
+    assert call(wsb=ws - 1) == 1                                        # workspace too small
+    assert call(workspace=ctypes.c_void_p(0x1010)) == 1                 # 256-byte aligned
+    assert call(q=null) == 1
+
 def test_noalloc_decode_checks_outputs_before_launching(b):
     # a misaligned or missing o_lat (or lse_out) is refused before the split-KV decode is
     # launched, so nothing touches a device
