@@ -285,6 +285,10 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
     uint32_t tcols = 32;
     while (tcols < static_cast<uint32_t>(a.NT)) tcols <<= 1;
 
+    // The weights are never written by an earlier kernel of the step, so the
+    // first stages' W tiles are requested before waiting for that kernel
+    // (programmatic dependent launch); the activations only after it.
+    const int npre = nkb < S ? nkb : S;
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
@@ -293,13 +297,20 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
         ptx::mbar_init(ptx::smem_u32(done), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
+        for (int kb = 0; kb < npre; ++kb) {
+            const uint32_t st = base + kb * stage_bytes;
+            const uint32_t fb = ptx::smem_u32(&full[kb]);
+            ptx::mbar_arrive_expect_tx(fb, stage_bytes);
+            ptx::tma_load_3d(st, &map_w, fb, m0, kb * 64, h);
+            ptx::tma_load_3d(st + 64 * 128, &map_w, fb, m0 + 64, kb * 64, h);
+        }
     }
     if (warp == 1) {
         ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
         ptx::tmem_relinquish<1>();
     }
     ptx::grid_dep_launch();
-    ptx::grid_dep_wait();   // global memory from here on
+    ptx::grid_dep_wait();   // other global memory from here on
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -317,9 +328,11 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
                     break;
                 const uint32_t st = base + s * stage_bytes;
                 const uint32_t fb = ptx::smem_u32(&full[s]);
-                ptx::mbar_arrive_expect_tx(fb, stage_bytes);
-                ptx::tma_load_3d(st, &map_w, fb, m0, kb * 64, h);
-                ptx::tma_load_3d(st + 64 * 128, &map_w, fb, m0 + 64, kb * 64, h);
+                if (kb >= npre) {   // (stages below npre: W requested before the dependency wait)
+                    ptx::mbar_arrive_expect_tx(fb, stage_bytes);
+                    ptx::tma_load_3d(st, &map_w, fb, m0, kb * 64, h);
+                    ptx::tma_load_3d(st + 64 * 128, &map_w, fb, m0 + 64, kb * 64, h);
+                }
                 ptx::tma_load_3d(st + kProjW, &map_x, fb, kb * 64, h, t0);
             }
             for (int k2 = (kb > S ? kb - S : 0); k2 < kb; ++k2)
@@ -472,13 +485,13 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     while (tcols < static_cast<uint32_t>(NT)) tcols <<= 1;
 
     ptx::grid_dep_launch();
-    ptx::grid_dep_wait();   // global memory from here on
     if (threadIdx.x == 0) {
         ptx::mbar_init(wfull, 1);
         ptx::mbar_init(done, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
-        // W_UV[h] rows [q * KC, (q + 1) * KC): issued first, lands during the merge
+        // W_UV[h] rows [q * KC, (q + 1) * KC): never written by an earlier kernel
+        // of the step, so requested before waiting for it; lands during the merge
         ptx::mbar_arrive_expect_tx(wfull, KB * 16384u);
         for (int kb = 0; kb < KB; ++kb) {
             const int k0 = static_cast<int>(q) * KC + kb * 64;
@@ -486,6 +499,7 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
             ptx::tma_load_3d(w_s + kb * 16384u + 8192u, &map_w, wfull, 64, k0, h);
         }
     }
+    ptx::grid_dep_wait();   // other global memory from here on
     if (warp == 1) {
         ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
         ptx::tmem_relinquish<1>();
