@@ -212,6 +212,7 @@ struct Misc {
     uint64_t seg_done;                // pair kernel: a segment's row sums and maxima are published
     float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
     uint64_t code_qk[pair::QK_STAGES], code_pv[pair::PV_STAGES];   // E4M3 pair kernel: codes landed
+    uint64_t kv_full[8], kv_empty[8];   // single kernel: its KV ring
 };
 static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
 
@@ -1032,7 +1033,10 @@ constexpr uint32_t Q_BYTES = Q_LAT + 2 * Q_ROPE;          // + zero K-chunk
 constexpr uint32_t ST_LAT = TOK * 128;                    // 16384
 constexpr uint32_t ST_ROPE = TOK * 16;                    // 2048
 constexpr uint32_t STAGE_BYTES = ST_LAT + 2 * ST_ROPE;    // 20480
-constexpr int STAGES = 2;
+#ifndef MLA_SINGLE_STAGES
+#define MLA_SINGLE_STAGES 4
+#endif
+constexpr int STAGES = MLA_SINGLE_STAGES;                 // KV ring depth (score and P buffers: 2)
 constexpr uint32_t P_BYTES = 2 * ROWS * 128;              // [128 rows x 128 tok] = 2 K-blocks
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_STAGE = 20480;                     // Q rounded up to 1 KB multiple
@@ -1045,10 +1049,12 @@ constexpr uint32_t TMEM_S = 128;                          // two 128-column scor
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16(128, TOK, 0, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(128, DC, 0, 1);
 static_assert(Q_BYTES <= OFF_STAGE, "q");
+static_assert(STAGES >= 2 && STAGES <= 8, "ring");
 static_assert(SMEM_BYTES <= 232448, "smem");
 static_assert((OFF_P % 1024) == 0 && (OFF_MISC % 1024) == 0, "align");
 }  // namespace single
 
+template <bool kSplit>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_single_kernel(const __grid_constant__ CUtensorMap map_ckv,
                          const __grid_constant__ CUtensorMap map_kr, const DecodeArgs args) {
@@ -1067,9 +1073,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     auto bar = [&](const uint64_t *b) { return ptx::smem_u32(b); };
 
     if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            ptx::mbar_init(bar(&misc->kv_full[i]), 1);
+            ptx::mbar_init(bar(&misc->kv_empty[i]), 1);
+        }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(bar(&misc->full[i]), 1);
-            ptx::mbar_init(bar(&misc->empty[i]), 1);
             ptx::mbar_init(bar(&misc->s_full[i]), 1);
             ptx::mbar_init(bar(&misc->s_free[i]), 4);
             ptx::mbar_init(bar(&misc->p_ready[i]), 4);
@@ -1141,16 +1149,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
                 const int32_t npages = (walk.L + 63) / 64;
                 for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
-                    const int s = static_cast<int>(k & 1);
+                    const int s = static_cast<int>(k % STAGES);
                     const int32_t p0 = static_cast<int32_t>(2 * t);
                     const bool two = p0 + 1 < npages;
                     int32_t pg[2] = {trow[p0], two ? trow[p0 + 1] : 0};
                     for (int i = 0; i < 2; ++i)
                         if (pg[i] < 0 || pg[i] >= args.num_pages) { bad_page = true; pg[i] = 0; }
-                    if (k >= 2 && !wait_bounded(bar(&misc->empty[s]), ((k >> 1) - 1) & 1,
-                                                abort_flag, args.timeout_ns))
+                    if (k >= STAGES && !wait_bounded(bar(&misc->kv_empty[s]), ((k / STAGES) - 1) & 1,
+                                                     abort_flag, args.timeout_ns))
                         break;
-                    const uint32_t fb = bar(&misc->full[s]);
+                    const uint32_t fb = bar(&misc->kv_full[s]);
                     const uint32_t npg = two ? 2u : 1u;
                     ptx::mbar_arrive_expect_tx(fb, npg * (64 * 128 + 64 * 16));
                     const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
@@ -1161,19 +1169,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 }
             }
             if (bad_page) record_error(kErrDeviceBounds);
-            for (int64_t kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk)
-                wait_bounded(bar(&misc->full[kk & 1]), (kk >> 1) & 1, abort_flag, args.timeout_ns);
+            for (int64_t kk = (k >= STAGES ? k - STAGES : 0); kk < k; ++kk)
+                wait_bounded(bar(&misc->kv_full[kk % STAGES]), (kk / STAGES) & 1, abort_flag, args.timeout_ns);
         }
     } else if (warp == 1) {
         if (ptx::elect_one()) {
             int64_t k = 0, g = 0;
             bool ok = true;
             auto issue_pv = [&](int64_t kp, bool first_of_seg) -> bool {
-                const int s = static_cast<int>(kp & 1);
+                const int s = static_cast<int>(kp & 1);            // P buffer
+                const int ks = static_cast<int>(kp % STAGES);      // KV stage
                 if (!wait_bounded(bar(&misc->p_ready[s]), (kp >> 1) & 1, abort_flag, args.timeout_ns))
                     return false;
                 ptx::tc_fence_after();
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint32_t st = base + OFF_STAGE + ks * STAGE_BYTES;
                 const uint32_t pbuf = base + OFF_P + s * P_BYTES;
                 for (int kk = 0; kk < TOK / 16; ++kk) {
                     const uint64_t a = ptx::smem_desc(pbuf + (kk >> 2) * (ROWS * 128) + (kk & 3) * 32,
@@ -1182,7 +1191,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     ptx::mma_bf16_ss<1>(tmem + TMEM_O, a, b, IDESC_PV,
                                         (first_of_seg && kk == 0) ? 0u : 1u);
                 }
-                ptx::mma_commit(bar(&misc->empty[s]));
+                ptx::mma_commit(bar(&misc->kv_empty[ks]));
                 ptx::mma_commit(bar(&misc->pv_done[s]));
                 return true;
             };
@@ -1190,8 +1199,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 const int64_t k0 = k;
                 if (!wait_bounded(bar(&misc->q_ready), g & 1, abort_flag, args.timeout_ns)) break;
                 for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
-                    const int s = static_cast<int>(k & 1);
-                    if (!wait_bounded(bar(&misc->full[s]), (k >> 1) & 1, abort_flag, args.timeout_ns)) {
+                    const int s = static_cast<int>(k & 1);             // score buffer
+                    const int ks = static_cast<int>(k % STAGES);       // KV stage
+                    if (!wait_bounded(bar(&misc->kv_full[ks]), (k / STAGES) & 1, abort_flag,
+                                      args.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -1201,7 +1212,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    const uint32_t st = base + OFF_STAGE + ks * STAGE_BYTES;
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t a = ptx::smem_desc(base + OFF_Q + kk * 32, 16, 1024,
                                                           ptx::kSwizzle128B);
@@ -1238,10 +1249,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             wait_bounded(bar(&misc->drain), 0, abort_flag, args.timeout_ns);
         }
     } else {
+        // kSplit (at most 64 query rows): query row r sits in MMA rows
+        // 32 (r / 16) + r % 16 and the same + 16, both TMEM lanes of one warp;
+        // the first lane takes the tile's tokens 0..63, the second 64..127, and
+        // the two meet by shuffles (row maximum per tile, sums and O at the
+        // end). Otherwise MMA row = query row and a lane takes all 128 tokens.
+        constexpr int TT = kSplit ? TOK / 2 : TOK;      // tokens per thread and tile
         const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;                 // query row = TMEM lane
+        const int tl = q4 * 32 + lane;                  // TMEM lane = MMA row
+        const int half = kSplit ? (lane >> 4) : 0;
+        const int row = kSplit ? 16 * q4 + (lane & 15) : tl;   // query row
         const bool real_row = row < args.rows;
-        const bool warp_real = (q4 * 32) < args.rows;   // warp holds at least one real row
+        const bool warp_real = (kSplit ? 16 * q4 : 32 * q4) < args.rows;   // warp holds a real row
         const int qi = real_row ? row / args.heads : 0;
         const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
         const int st_tid = threadIdx.x - kSoftmaxWarp0 * 32;
@@ -1251,7 +1270,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         };
         auto load_q = [&](int32_t b) {   // all of a thread's loads in flight at once
             const __nv_bfloat16 *qb = args.q + static_cast<int64_t>(b) * args.rows * D;
-            constexpr int NQ = ROWS * (D / 8) / 128;   // 9 chunks per thread
+            constexpr int QR = kSplit ? ROWS / 2 : ROWS;              // query rows held
+            constexpr int NQ = (QR * (D / 8) + 127) / 128;           // chunks per thread
             uint4 v[NQ];
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
@@ -1264,12 +1284,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
                 const int idx = st_tid + 128 * i;
+                if (idx >= QR * (D / 8)) break;
                 const int r = idx / (D / 8);
                 const int cc = idx - r * (D / 8);
-                uint32_t dst;
-                if (cc < 8) dst = base + OFF_Q + sw128(r, cc);
-                else dst = base + OFF_Q + Q_LAT + (r >> 3) * 128 + (r & 7) * 16;
-                st_shared_v4(dst, v[i].x, v[i].y, v[i].z, v[i].w);
+#pragma unroll
+                for (int dup = 0; dup < (kSplit ? 2 : 1); ++dup) {
+                    const int m = kSplit ? 32 * (r >> 4) + (r & 15) + 16 * dup : r;   // MMA row
+                    uint32_t dst;
+                    if (cc < 8) dst = base + OFF_Q + sw128(m, cc);
+                    else dst = base + OFF_Q + Q_LAT + (m >> 3) * 128 + (m & 7) * 16;
+                    st_shared_v4(dst, v[i].x, v[i].y, v[i].z, v[i].w);
+                }
             }
             ptx::fence_proxy_async_smem();
             arrive(&misc->q_ready);
@@ -1293,15 +1318,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     break;
                 }
                 ptx::tc_fence_after();
-                float v[TOK];
+                float v[TT];
                 if (warp_real) {
+                    // (a tensor-memory load takes one column address for the whole
+                    // warp: with kSplit every lane loads both halves and keeps its own)
 #pragma unroll
-                    for (int c = 0; c < TOK / 32; ++c) {
+                    for (int c = 0; c < TT / 32; ++c) {
                         uint32_t sr[32];
                         ptx::tmem_ld32(tmem + lane_base + TMEM_S + TOK * s + 32 * c, sr);
-                        ptx::tmem_wait_ld();
+                        if (kSplit) {
+                            uint32_t sr2[32];
+                            ptx::tmem_ld32(tmem + lane_base + TMEM_S + TOK * s + TT + 32 * c, sr2);
+                            ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[32 * c + j] = __uint_as_float(sr[j]);
+                            for (int j = 0; j < 32; ++j) v[32 * c + j] = __uint_as_float(half ? sr2[j] : sr[j]);
+                        } else {
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[32 * c + j] = __uint_as_float(sr[j]);
+                        }
                     }
                 }
                 ptx::tc_fence_before();
@@ -1309,12 +1344,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
                 float alpha = 1.f;
                 if (warp_real) {
-                    const int32_t tok0 = static_cast<int32_t>(t) * TOK;
-                    if (tok0 + TOK > vis) {   // mask the tokens this row does not see
+                    const int32_t tok0 = static_cast<int32_t>(t) * TOK + TT * half;
+                    if (tok0 + TT > vis) {   // mask the tokens this row does not see
 #pragma unroll
-                        for (int j = 0; j < TOK; ++j) v[j] = (tok0 + j < vis) ? v[j] : -INFINITY;
+                        for (int j = 0; j < TT; ++j) v[j] = (tok0 + j < vis) ? v[j] : -INFINITY;
                     }
-                    const float mx = max_of<TOK>(v);
+                    float mx = max_of<TT>(v);
+                    if (kSplit) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));   // the row's two halves
                     if (mx > -INFINITY && (m_run == -INFINITY ||
                                            (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
                         alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - mx) * args.scale_log2);
@@ -1323,11 +1359,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
                     float psum = 0.f;
 #pragma unroll
-                    for (int j = 0; j < TOK; ++j) {
+                    for (int j = 0; j < TT; ++j) {
                         v[j] = exp2f(fmaf(v[j], args.scale_log2, -mb));
                         psum += v[j];
                     }
-                    l_run = fmaf(l_run, alpha, psum);
+                    l_run = fmaf(l_run, alpha, psum);   // (kSplit: this half's share)
                 }
                 const bool need = warp_real && (k > k0) && (alpha != 1.f);
                 if (__any_sync(0xffffffffu, need)) {
@@ -1359,10 +1395,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                     }
                 }
                 if (warp_real) {
-                    const uint32_t pb = base + OFF_P + s * P_BYTES;
+                    // this thread's tokens of MMA row tl (kSplit: one 64-token K block;
+                    // the other block of the row keeps the zeros written at start)
+                    const uint32_t pb = base + OFF_P + s * P_BYTES + half * (ROWS * 128);
 #pragma unroll
-                    for (int c = 0; c < TOK / 8; ++c) {
-                        st_shared_v4(pb + (c >> 3) * (ROWS * 128) + sw128(row, c & 7),
+                    for (int c = 0; c < TT / 8; ++c) {
+                        st_shared_v4(pb + (c >> 3) * (ROWS * 128) + sw128(tl, c & 7),
                                      pack_bf16x2(v[8 * c + 0], v[8 * c + 1]),
                                      pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
                                      pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
@@ -1376,7 +1414,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 // reading the stage (s_full) and P.V waits for p_ready.
                 const int32_t valid = L - static_cast<int32_t>(t) * TOK;
                 if (valid < TOK) {
-                    const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                    const uint32_t st = base + OFF_STAGE + static_cast<int>(k % STAGES) * STAGE_BYTES;
                     for (int idx = st_tid; idx < (TOK - valid) * 8; idx += 128)
                         st_shared_v4(st + (valid + (idx >> 3)) * 128 + (idx & 7) * 16, 0u, 0u, 0u, 0u);
                 }
@@ -1393,14 +1431,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 break;
             ptx::tc_fence_after();
             if (warp_real) {
-                const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                // kSplit: the row's sum and O are its two lanes' shares added (the
+                // same sum in both lanes); each lane writes one 32-channel half
+                const float l_row = kSplit ? l_run + __shfl_xor_sync(0xffffffffu, l_run, 16) : l_run;
+                const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
                 float *dst = args.o_part + (slot * args.rows + row) * DC;
 #pragma unroll 1
                 for (int cch = 0; cch < DC / 32; ++cch) {
                     uint32_t o[32];
                     ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * cch, o);
                     ptx::tmem_wait_ld();
-                    if (real_row) {
+                    if (kSplit) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float mine = __uint_as_float(o[j]);
+                            const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+                            o[j] = __float_as_uint(half ? other + mine : mine + other);   // lane order: tokens 0..63 first
+                        }
+                    }
+                    if (real_row && (!kSplit || cch == half)) {
                         float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cch);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
@@ -1410,9 +1459,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                                 __uint_as_float(o[4 * j + 3]) * inv);
                     }
                 }
-                if (real_row)
+                if (real_row && half == 0)
                     args.lse_part[slot * args.rows + row] =
-                        (l_run > 0.f) ? m_run * args.scale + logf(l_run) : -INFINITY;
+                        (l_row > 0.f) ? m_run * args.scale + logf(l_row) : -INFINITY;
             }
             ptx::tc_fence_before();
             arrive(&misc->o_free);

@@ -81,7 +81,10 @@ mla_status device_ready() {
                                  mla::pair::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::pair::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::decode_single_kernel,
+            cudaFuncSetAttribute(mla::decode_single_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mla::single::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_single_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::single::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -115,7 +118,9 @@ mla_status device_ready() {
                                  carve) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_pair_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  carve) != cudaSuccess ||
-            cudaFuncSetAttribute(mla::decode_single_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+            cudaFuncSetAttribute(mla::decode_single_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carve) != cudaSuccess ||
+            cudaFuncSetAttribute(mla::decode_single_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  carve) != cudaSuccess) {
             st.status = MLA_ERR_CUDA;
             return;
@@ -491,8 +496,11 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
             return st;
         if ((st = pool_map(&mkr, kr, 8, num_pages, 8, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != MLA_OK)
             return st;
-        return launch_pdl(mla::decode_single_kernel, dim3(num_parts), dim3(mla::kDecodeThreads),
-                          mla::single::SMEM_BYTES, s, mc, mkr, a);
+        // at most 64 query rows: each row on two TMEM lanes, half the tile's tokens each
+        return a.rows <= 64 ? launch_pdl(mla::decode_single_kernel<true>, dim3(num_parts), dim3(mla::kDecodeThreads),
+                                         mla::single::SMEM_BYTES, s, mc, mkr, a)
+                            : launch_pdl(mla::decode_single_kernel<false>, dim3(num_parts),
+                                         dim3(mla::kDecodeThreads), mla::single::SMEM_BYTES, s, mc, mkr, a);
     }
 }
 

@@ -163,6 +163,13 @@ def test_parity_retrofit(api):
     _parity(api, workload("retrofit"), 16)
 
 
+@pytest.mark.parametrize("heads", [40, 64])
+def test_parity_retrofit_more_than_64_rows(api, heads):
+    # n_q * heads = 80 and 128 query rows: one TMEM lane per row (at most 64 rows
+    # put each row on two lanes that split the tile's tokens)
+    _parity(api, workload("retrofit", batch=3, heads=heads, seq_len=700), 8)
+
+
 def test_parity_long_context(api):
     r, inp = _parity(api, workload("long"), 8)
     # the fused combine + absorb-out on the same full-size partials (the bench's step)
