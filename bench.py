@@ -55,7 +55,12 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM bytes per launch of the decode kernel from an ncu capture, keyed by
 # (sha256 of the kernel source it was taken on, workload, cache format);
 # reported only while the source is unchanged.
-TRAFFIC = {}
+TRAFFIC = {
+    # decode_pair_kernel<false>, long (B16 L65536): 1,213,082,112 read + 7,461,120 written
+    ('edb870d707fcedb1', "long", "bf16"): 1220543232,
+    # decode_pair_kernel<true>, long, E4M3 cache: 679,816,192 read + 7,271,936 written
+    ('edb870d707fcedb1', "long", "fp8"): 687088128,
+}
 
 
 def _args():
