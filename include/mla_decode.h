@@ -95,8 +95,11 @@ mla_status mla_absorb_q(const mla_dims *dims, const void *q_c, const void *q_r, 
                         void *q_out, int32_t num_tokens, void *stream);
 
 /* Number of cache partitions mla_decode_splitkv should use for a batch whose
- * sequences hold total_tiles 64-token tiles in all (sum of ceil(L_b / 64)),
- * on a device with num_sms multiprocessors. Host-only arithmetic; returns >= 1. */
+ * sequences hold total_tiles tiles in all (sum of ceil(L_b / tile), tile = 64
+ * tokens for d_latent 512, 128 for d_latent 64), on a device with num_sms
+ * multiprocessors: min(ceil(total_tiles / 8), num_sms / 2) for d_latent 512
+ * (at most one per CTA pair), min(total_tiles, num_sms) for d_latent 64.
+ * Host-only arithmetic; returns >= 1. */
 int32_t mla_decode_num_parts(const mla_dims *dims, int64_t total_tiles, int32_t num_sms);
 
 /* Bytes of device workspace mla_decode_splitkv / mla_combine need for `batch`

@@ -53,18 +53,18 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// Bounded spin until the shared-memory word at `slot` carries `tag` in its low
-// 8 bits; the word is returned in *out. False after a timeout (abort raised).
+// Bounded spin until the shared-memory word at `slot` carries `tag` in its
+// lowest bit; the word is returned in *out. False after a timeout (abort raised).
 __device__ __forceinline__ bool wait_word(const uint32_t *slot, uint32_t tag,
                                           volatile int32_t *abort_flag, int64_t timeout_ns,
                                           uint32_t *out) {
     const volatile uint32_t *vs = slot;
     uint32_t v = *vs;
-    if ((v & 0xFFu) == tag) { *out = v; return true; }
+    if ((v & 1u) == tag) { *out = v; return true; }
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         v = *vs;
-        if ((v & 0xFFu) == tag) { *out = v; return true; }
+        if ((v & 1u) == tag) { *out = v; return true; }
         if ((it & 15u) == 0u) {
             if (*abort_flag) return false;
             if (static_cast<int64_t>(ptx::globaltimer_ns() - t0) > timeout_ns) {

@@ -207,7 +207,7 @@ struct Misc {
     int32_t pad0;
     int64_t cur_O, cur_S, cur_N, cur_P;   // plan: cost offset, slot base, total cost, partitions
     uint32_t xtag[2][128];            // pair kernel: tagged half-row maxima, by tile parity
-    uint32_t xltag[128];              // pair kernel: tagged half-row sums, per segment
+    uint32_t xltag[128];              // pair kernel: tagged half-row sums, by segment
     uint64_t q_free;                  // pair kernel: the last QK^T of a segment is done (Q may be replaced)
     uint64_t seg_done;                // pair kernel: a segment's row sums and maxima are published
     float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
@@ -400,7 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         ptx::fence_mbar_init();
     }
     for (int i = threadIdx.x; i < 3 * 128; i += blockDim.x)
-        (i < 256 ? misc->xtag[i >> 7][i & 127] : misc->xltag[i - 256]) = 0u;
+        (i < 256 ? misc->xtag[i >> 7][i & 127] : misc->xltag[i - 256]) = 1u;   // tag of "use -1"
     if (warp == 1) {
         ptx::tmem_alloc<2>(bar(reinterpret_cast<uint64_t *>(&misc->tmem_base)), TMEM_COLS);
         ptx::tmem_relinquish<2>();
@@ -897,17 +897,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
                     for (int j = 0; j < 32; ++j) v[j] = (tok0 + j < vis) ? __uint_as_float(sr[j]) : -INFINITY;
                 }
                 float mx = max_of<32>(v);
-                // half-row maxima meet through tagged words: low 8 mantissa bits
-                // carry the tile tag, both lanes use the same truncated values
-                const uint32_t tag = static_cast<uint32_t>((k >> 1) % 255) + 1u;
-                const uint32_t mine = (__float_as_uint(mx) & 0xFFFFFF00u) | tag;
+                // Half-row maxima meet through tagged words: the lowest mantissa
+                // bit carries the parity of the word's use (k / 2); a lane cannot
+                // be two uses ahead of its partner's read (it needs the partner's
+                // word of every tile in between), so one bit tells the uses apart.
+                // Both lanes use the same two values with that bit cleared (1 ulp,
+                // so the exponentials stay finite for scores up to ~2^23 / scale_log2).
+                const uint32_t tag = static_cast<uint32_t>((k >> 1) & 1);
+                const uint32_t mine = (__float_as_uint(mx) & ~1u) | tag;
                 reinterpret_cast<volatile uint32_t *>(misc->xtag[s])[lt] = mine;
                 uint32_t other = 0;
                 if (!wait_word(&misc->xtag[s][lt ^ 64], tag, abort_flag, args.timeout_ns, &other)) {
                     ok = false;
                     break;
                 }
-                mx = fmaxf(__uint_as_float(mine & 0xFFFFFF00u), __uint_as_float(other & 0xFFFFFF00u));
+                mx = fmaxf(__uint_as_float(mine & ~1u), __uint_as_float(other & ~1u));
 
                 float alpha = 1.f;
                 if (mx > -INFINITY && (m_run == -INFINITY ||
@@ -991,15 +995,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
 
             // the segment's row sum: both halves of the row meet; published with
             // the running maximum for the segment warps' epilogue
-            const uint32_t ltag = static_cast<uint32_t>(seg_no % 255) + 1u;
+            const uint32_t ltag = static_cast<uint32_t>(seg_no & 1);   // (as above, by segment)
             const int gpar = static_cast<int>(seg_no & 1);
             ++seg_no;
-            const uint32_t lmine = (__float_as_uint(l_run) & 0xFFFFFF00u) | ltag;
+            const uint32_t lmine = (__float_as_uint(l_run) & ~1u) | ltag;
             reinterpret_cast<volatile uint32_t *>(misc->xltag)[lt] = lmine;
             uint32_t lother = 0;
             if (!wait_word(&misc->xltag[lt ^ 64], ltag, abort_flag, args.timeout_ns, &lother)) break;
             // identical in both lanes: the same two truncated terms, added commutatively
-            const float l_row = __uint_as_float(lmine & 0xFFFFFF00u) + __uint_as_float(lother & 0xFFFFFF00u);
+            const float l_row = __uint_as_float(lmine & ~1u) + __uint_as_float(lother & ~1u);
             if (half == 0) {
                 misc->seg_l[gpar][row] = l_row;
                 misc->seg_m[gpar][row] = m_run;

@@ -115,7 +115,11 @@ def test_plan_matches_brute_force(b, latent):
 def test_num_parts_and_workspace(b):
     d = _dims(b)
     lib = b.lib
-    assert lib.mla_decode_num_parts(ctypes.byref(d), 4, 148) == 1
+    assert lib.mla_decode_num_parts(ctypes.byref(d), 4, 148) == 1       # at least 8 tiles each
+    assert lib.mla_decode_num_parts(ctypes.byref(d), 100, 148) == 13
+    small = _dims(b, n_q=2, num_heads=32, d_nope=120, d_latent=64, d_rope=8)
+    assert lib.mla_decode_num_parts(ctypes.byref(small), 100, 148) == 100   # one per SM at most
+    assert lib.mla_decode_num_parts(ctypes.byref(small), 1000, 148) == 148
     assert lib.mla_decode_num_parts(ctypes.byref(d), 16 * 1024, 148) == 74
     assert lib.mla_decode_num_parts(ctypes.byref(d), 0, 148) == 1
     ws = lib.mla_decode_workspace_bytes(ctypes.byref(d), 16, 74)

@@ -181,3 +181,34 @@ def test_decode_fp8_long_context_sampled(api):
                                               scale)
         _check(_f64(o8[b:b + 1]), o_ref, f"long b={b}")
         assert np.abs(_f64(lse8[b:b + 1]) - lse_ref).max() <= 1e-3
+
+
+@pytest.mark.parametrize("n_q", [1, 2])
+def test_decode_fp8_extreme_scales_bitwise(api, n_q):
+    # codes and per-token scales written directly (not through the quantiser): scales
+    # from 2^-140 (products below the fp32 normal range) to 2^12 (scores ~1e8), random
+    # non-NaN codes, and n_q = 2 (causal pair).
+    # The decode must equal the bf16 decode on the oracle's dequantisation of the
+    # same codes bit for bit: the same operands reach the same products.
+    w = workload("dsv3", batch=3, heads=16, n_q=n_q, ragged=(2, 700), seq_len=0)
+    inp = make_inputs(w, seed=47, seq_lens=(2, 333, 700))
+    d = to_device(inp, "cuda")
+    dims = api.dims_for(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"])
+    pages = inp["ckv_pool"].shape[0]
+    g = torch.Generator().manual_seed(48)
+    codes = torch.randint(0, 256, (pages, 64, 512), generator=g, dtype=torch.int32).to(torch.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x7E                              # no NaN codes
+    expo = torch.randint(-140, 13, (pages, 64), generator=g).to(torch.float32)
+    scales = torch.ldexp(1.0 + torch.rand(pages, 64, generator=g), expo).to(torch.float32)
+    deq = oracle.bf16_from_bits(oracle.dequant_fp8_rows(codes.numpy(), scales.numpy()))
+    pool_d = deq.cuda()
+    codes_d, scales_d = codes.cuda(), scales.cuda()
+    q = api.absorb_q(d["q_c"], d["q_r"], d["w_uk"], dims)
+    for parts in (None, 3):
+        P = _parts(api, dims, inp) if parts is None else parts
+        o8, lse8 = _decode_fp8(api, d, q, codes_d, scales_d, d["kr_pool"], dims, P)
+        ws = api.decode_splitkv(q, pool_d, d["kr_pool"], d["block_table"], d["seq_lens"], dims, P)
+        o16, lse16 = api.combine(ws, d["seq_lens"], d["block_table"].shape[1], dims, P)
+        torch.cuda.synchronize()
+        assert api.get_device_error() == 0
+        assert torch.equal(o8, o16) and torch.equal(lse8, lse16), P
