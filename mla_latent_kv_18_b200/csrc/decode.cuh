@@ -126,8 +126,13 @@ struct SegmentWalker {
     // current segment
     int32_t seg_b, L;
     int64_t t_begin, t_end, slot;
+    bool primed = false;   // the current segment was found ahead: next() hands it out
 
     __device__ bool next() {
+        if (primed) {
+            primed = false;
+            return true;
+        }
         while (tile < te && b < batch) {
             bool bad = false;
             const int32_t Lb = clamp_len(seq_lens[b], max_pages, n_q, &bad);
@@ -177,6 +182,15 @@ constexpr uint32_t MISC_BYTES = 3072;
 constexpr uint32_t OFF_EPI = OFF_MISC + MISC_BYTES;         // partial-store staging, 1 KB per segment warp
 constexpr uint32_t EPI_BYTES = 4 * 32 * 32;
 constexpr uint32_t SMEM_BYTES = OFF_EPI + EPI_BYTES;     // dynamic smem base is 1 KB aligned
+// The first segment's Q blocks 0..QT-1 land here by TMA before they are copied to
+// tensor memory: P.V slot 1 and P buffer 0, which nothing uses until Q is ready
+// (the P.V producer waits for q_stage_free before its first copy into slot 1).
+constexpr uint32_t OFF_QSTAGE = OFF_PV + STAGE_PV;
+// The first segment's first FIRST_PAGES page numbers, read with the plan, wait in
+// the partial-store staging tile: the producers read them at once after setup,
+// and the segment warps first write there at that segment's end.
+constexpr int FIRST_PAGES = 4;
+constexpr uint32_t OFF_FIRST_PAGES = OFF_EPI;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 0;                 // two 128-column accumulators (c = 0, 1)
 constexpr uint32_t TMEM_S = 256;               // three 32-column score buffers
@@ -190,6 +204,7 @@ constexpr uint32_t CODE_BYTES = 16384;         // QK^T: 32 tokens x 512; P.V: 64
 constexpr uint32_t SC_BYTES = 4 * 32 * 4;      // four copies of 32 tokens' scales per slot
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(TMEM_Q + QT * 32 <= TMEM_COLS, "tensor memory budget");
+static_assert(PV_STAGES == 2 && OFF_QSTAGE + QT * ROWS_CTA * 128 <= OFF_P + P_BYTES, "Q staging");
 static_assert((OFF_QK % 1024) == 0 && (OFF_PV % 1024) == 0 && (OFF_P % 1024) == 0 &&
                   (OFF_MISC % 1024) == 0, "align");
 }  // namespace pair
@@ -213,6 +228,12 @@ struct Misc {
     float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
     uint64_t code_qk[pair::QK_STAGES], code_pv[pair::PV_STAGES];   // E4M3 pair kernel: codes landed
     uint64_t kv_full[8], kv_empty[8];   // single kernel: its KV ring
+    // pair kernel: the partition's first segment, found before the dependency
+    // wait (the walker's state after its first next(); first_b < 0: none)
+    int64_t first_tile, first_slot;
+    int32_t first_b, first_L, first_t_begin, first_t_end;
+    uint64_t q_tma;                   // pair kernel: the first segment's Q has landed
+    uint64_t q_stage_free;            // pair kernel: its staged blocks are in tensor memory
 };
 static_assert(sizeof(Misc) <= pair::MISC_BYTES, "misc");
 
@@ -349,7 +370,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
     decode_pair_kernel(const __grid_constant__ CUtensorMap map_ckv32,
                        const __grid_constant__ CUtensorMap map_ckv64,
                        const __grid_constant__ CUtensorMap map_kr32,
-                       const __grid_constant__ CUtensorMap map_sc, const DecodeArgs args) {
+                       const __grid_constant__ CUtensorMap map_sc,
+                       const __grid_constant__ CUtensorMap map_q, const DecodeArgs args) {
     using namespace pair;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = ptx::smem_u32(smem_raw);
@@ -396,6 +418,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         ptx::mbar_init(bar(&misc->drain), 1);
         ptx::mbar_init(bar(&misc->q_free), 1);      // multicast commit from the leader
         ptx::mbar_init(bar(&misc->seg_done), 4);    // 4 softmax warps
+        ptx::mbar_init(bar(&misc->q_tma), 1);
+        ptx::mbar_init(bar(&misc->q_stage_free), 4);   // this CTA's 4 segment warps
         misc->abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -406,7 +430,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         ptx::tmem_relinquish<2>();
     }
     ptx::grid_dep_launch();
-    ptx::grid_dep_wait();   // global memory from here on
+    // The plan reads only the sequence lengths, which no kernel of a decode step
+    // writes (the kernel ahead on the stream produces q): it is made, down to
+    // this partition's first segment, before waiting for that kernel.
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, -1);
@@ -414,18 +440,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
         const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, ts);
+        SegmentWalker w0;
+        w0.seq_lens = args.seq_lens;
+        w0.batch = args.batch;
+        w0.max_pages = args.max_pages;
+        w0.n_q = args.n_q;
+        w0.tile_tokens = TOK;
+        w0.N = N;
+        w0.P = c.parts;
+        w0.p = part;
+        w0.b = s.b;
+        w0.O = s.cost_off;
+        w0.S = s.slot_base;
+        w0.tile = (part < c.parts) ? part_start(part, N, c.parts) : 0;
+        w0.te = (part < c.parts) ? part_start(part + 1, N, c.parts) : 0;
+        const bool have0 = w0.next();
         if (lane == 0) {
-            misc->cur_b = s.b;
-            misc->cur_O = s.cost_off;
-            misc->cur_S = s.slot_base;
+            misc->cur_b = w0.b;
+            misc->cur_O = w0.O;
+            misc->cur_S = w0.S;
             misc->cur_N = N;
             misc->cur_P = c.parts;
+            misc->first_tile = w0.tile;
+            misc->first_slot = have0 ? w0.slot : 0;
+            misc->first_b = have0 ? w0.seg_b : -1;
+            misc->first_L = have0 ? w0.L : 0;
+            misc->first_t_begin = have0 ? static_cast<int32_t>(w0.t_begin) : 0;
+            misc->first_t_end = have0 ? static_cast<int32_t>(w0.t_end) : 0;
+            if (have0) {   // the first page numbers, for the producers
+                const int32_t *trow0 = args.block_table + static_cast<int64_t>(w0.seg_b) * args.max_pages;
+                int32_t *pg = reinterpret_cast<int32_t *>(smem + OFF_FIRST_PAGES);
+#pragma unroll
+                for (int i = 0; i < FIRST_PAGES; ++i)
+                    pg[i] = (w0.t_begin + i < w0.t_end) ? trow0[w0.t_begin + i] : 0;
+            }
             ptx::prefetch_tensormap(&map_ckv32);
             ptx::prefetch_tensormap(&map_ckv64);
             ptx::prefetch_tensormap(&map_kr32);
+            ptx::prefetch_tensormap(&map_q);
             if (kFp8) ptx::prefetch_tensormap(&map_sc);
         }
     }
+    ptx::grid_dep_wait();   // other global memory from here on
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync();
@@ -444,12 +500,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
     walk.b = misc->cur_b;
     walk.O = misc->cur_O;
     walk.S = misc->cur_S;
-    if (part < walk.P) {
-        walk.tile = part_start(part, walk.N, walk.P);
-        walk.te = part_start(part + 1, walk.N, walk.P);
-    } else {
-        walk.tile = walk.te = 0;   // idle partition
-    }
+    walk.te = (part < walk.P) ? part_start(part + 1, walk.N, walk.P) : 0;   // 0: idle partition
+    walk.tile = misc->first_tile;
+    walk.primed = misc->first_b >= 0;
+    walk.seg_b = misc->first_b;
+    walk.L = misc->first_L;
+    walk.t_begin = misc->first_t_begin;
+    walk.t_end = misc->first_t_end;
+    walk.slot = misc->first_slot;
 
     if (warp == 0 || warp == 6) {
         // ------------------------------------------------------ TMA producers
@@ -467,15 +525,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
             const uint32_t tx = kFp8 ? 2 * (OWN * 128) : 2 * (qk ? STAGE_QK : STAGE_PV);
             int64_t k = 0;
             bool bad_page = false;
-            while (!*abort_flag && walk.next()) {
+            if (qk && walk.primed) {
+                // the first segment's Q: blocks 0..QT-1 to the staging area (the
+                // segment warps move them to tensor memory), the rest to their place
+                const uint32_t qbar = bar(&misc->q_tma);
+                ptx::mbar_arrive_expect_tx(qbar, NB * ROWS_CTA * 128);
+                for (int j = 0; j < NB; ++j)
+                    ptx::tma_load_3d(j < QT ? base + OFF_QSTAGE + j * (ROWS_CTA * 128)
+                                            : base + OFF_Q + (j - QT) * (ROWS_CTA * 128),
+                                     &map_q, qbar, 64 * j, ROWS_CTA * static_cast<int>(rank), walk.seg_b);
+            }
+            bool first_seg = walk.primed;
+            for (; !*abort_flag && walk.next(); first_seg = false) {
                 const int32_t *trow = args.block_table + static_cast<int64_t>(walk.seg_b) * args.max_pages;
                 for (int64_t t = walk.t_begin; t < walk.t_end; ++t, ++k) {
                     const int s = static_cast<int>(k % nst);
                     const int64_t use = k / nst;
-                    int32_t page = trow[t];
+                    // the first tiles' pages were read with the plan (k counts the
+                    // first segment's tiles first)
+                    int32_t page = (first_seg && k < FIRST_PAGES)
+                                       ? reinterpret_cast<const int32_t *>(smem + OFF_FIRST_PAGES)[k]
+                                       : trow[t];
                     if (page < 0 || page >= args.num_pages) { bad_page = true; page = 0; }
                     if (use >= 1 && !wait_bounded(bar(&emptyb[s]), (use - 1) & 1, abort_flag,
                                                   args.timeout_ns))
+                        break;
+                    if (!qk && k == 1 &&   // slot 1 held the first segment's staged Q
+                        !wait_bounded(bar(&misc->q_stage_free), 0, abort_flag, args.timeout_ns))
                         break;
                     const uint32_t fb = (rank == 0) ? bar(&fullb[s]) : leader_bar(&fullb[s]);
                     if constexpr (kFp8) {
@@ -764,6 +840,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
             arrive_leader(&misc->q_ready);
         };
 
+        // The first segment's Q, landed by TMA: blocks QT..8 are in place,
+        // blocks 0..QT-1 (128-byte swizzled rows) are copied to tensor memory.
+        auto load_q_staged = [&]() {
+            if (wait_bounded(bar(&misc->q_tma), 0, abort_flag, args.timeout_ns)) {
+#pragma unroll 1
+                for (int j = 0; j < QT; ++j) {
+                    uint32_t w[32];
+                    const uint32_t src = base + OFF_QSTAGE + j * (ROWS_CTA * 128);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint4 v = ld_shared_v4(src + sw128(row, i));
+                        w[4 * i] = v.x;
+                        w[4 * i + 1] = v.y;
+                        w[4 * i + 2] = v.z;
+                        w[4 * i + 3] = v.w;
+                    }
+                    ptx::tmem_st32(tmem + lane_base + TMEM_Q + 32 * j, w);
+                }
+            }
+            ptx::tmem_wait_st();
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(&misc->q_stage_free));
+            arrive_leader(&misc->q_ready);
+        };
+
         auto prefetch_q = [&](int32_t b) {   // the next segment's Q rows into L2
             if (!real_row || half) return;
             const char *qrow = reinterpret_cast<const char *>(
@@ -776,7 +879,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         int64_t k = 0;
         int64_t g = 0;
         bool have = walk.next();
-        if (have) load_q(walk.seg_b);
+        if (have) load_q_staged();
         while (have && !*abort_flag) {
             const int64_t slot = walk.slot;
             const int64_t kl = k + (walk.t_end - walk.t_begin) - 1;   // the segment's last tile

@@ -444,6 +444,14 @@ mla::DecodeArgs decode_args(const mla_dims *dims, const void *q, int32_t num_pag
     return a;
 }
 
+// q [batch, rows, 576] bf16 as [64 rows x 64 channels] boxes (128-byte swizzled):
+// the pair kernel's TMA copy of a segment's Q; rows past `rows` read as zeros.
+mla_status q_map(CUtensorMap *m, const void *q, const mla_dims *dims, int32_t batch) {
+    const uint64_t D = static_cast<uint64_t>(dims->d_latent + dims->d_rope);
+    const uint64_t R = static_cast<uint64_t>(dims->n_q) * dims->num_heads;
+    return map_3d(m, q, D, R, static_cast<uint64_t>(batch), D * 2, R * D * 2, 64, mla::pair::ROWS_CTA, 1);
+}
+
 mla_status check_decode_common(const mla_dims *dims, const void *q, int32_t num_pages,
                                const int32_t *block_table, int32_t max_pages_per_seq,
                                const int32_t *seq_lens, int32_t batch, int32_t num_parts,
@@ -492,8 +500,10 @@ mla_status mla_decode_splitkv(const mla_dims *dims, const void *q, const mla_poo
         if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
             return st;
+        CUtensorMap mq;
+        if ((st = q_map(&mq, q, dims, batch)) != MLA_OK) return st;
         return launch_pdl(mla::decode_pair_kernel<false>, dim3(2 * num_parts), dim3(mla::kPairThreads),
-                          mla::pair::SMEM_BYTES, s, m32, m64, mkr, mkr /* no scales */, a);
+                          mla::pair::SMEM_BYTES, s, m32, m64, mkr, mkr /* no scales */, mq, a);
     } else {
         CUtensorMap mc, mkr;
         if ((st = pool_map(&mc, ckv, 64, num_pages, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
@@ -536,8 +546,10 @@ mla_status mla_decode_splitkv_fp8(const mla_dims *dims, const void *q, const mla
     if ((st = pool_map(&mkr, kr, 64, num_pages, 64, mla::pair::OWN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
         return st;
     if ((st = scale_map(&msc, scales, num_pages, 32)) != MLA_OK) return st;
+    CUtensorMap mq;
+    if ((st = q_map(&mq, q, dims, batch)) != MLA_OK) return st;
     return launch_pdl(mla::decode_pair_kernel<true>, dim3(2 * num_parts), dim3(mla::kPairThreadsFp8),
-                      mla::pair::SMEM_BYTES, static_cast<cudaStream_t>(stream), mc, mc, mkr, msc, a);
+                      mla::pair::SMEM_BYTES, static_cast<cudaStream_t>(stream), mc, mc, mkr, msc, mq, a);
 }
 
 mla_status mla_combine(const mla_dims *dims, const void *workspace, size_t workspace_bytes,
