@@ -37,13 +37,14 @@
  *   - Kernels are launched with programmatic dependent launch: each may start
  *     while the kernel ahead of it on the stream is still running, and waits
  *     for that kernel to finish before it reads that kernel's outputs. The
- *     decode calls read seq_lens and block_table before that wait; the other
- *     calls read only their weights before it. The kernels of this library
- *     never write those inputs, so a stream that produces them with copies,
- *     with this library's calls or with kernels that do not trigger their
- *     dependents early is always safe; a custom kernel that triggers early
- *     (griddepcontrol.launch_dependents) must not write a decode call's
- *     seq_lens or block_table when it runs directly before that call.
+ *     decode calls read seq_lens and block_table before that wait, the
+ *     combine calls seq_lens; the other calls read only their weights before
+ *     it. The kernels of this library never write those inputs, so a stream
+ *     that produces them with copies, with this library's calls or with
+ *     kernels that do not trigger their dependents early is always safe; a
+ *     custom kernel that triggers early (griddepcontrol.launch_dependents)
+ *     must not write a call's seq_lens or block_table when it runs directly
+ *     before that call.
  */
 #ifndef MLA_DECODE_H
 #define MLA_DECODE_H

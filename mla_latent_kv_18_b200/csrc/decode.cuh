@@ -228,8 +228,8 @@ struct Misc {
     float seg_l[2][64], seg_m[2][64]; // pair kernel: those sums and maxima, by segment parity
     uint64_t code_qk[pair::QK_STAGES], code_pv[pair::PV_STAGES];   // E4M3 pair kernel: codes landed
     uint64_t kv_full[8], kv_empty[8];   // single kernel: its KV ring
-    // pair kernel: the partition's first segment, found before the dependency
-    // wait (the walker's state after its first next(); first_b < 0: none)
+    // the partition's first segment, found before the dependency wait (the
+    // walker's state after its first next(); first_b < 0: none)
     int64_t first_tile, first_slot;
     int32_t first_b, first_L, first_t_begin, first_t_end;
     uint64_t q_tma;                   // pair kernel: the first segment's Q has landed
@@ -1206,7 +1206,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         ptx::tmem_relinquish<1>();
     }
     ptx::grid_dep_launch();
-    ptx::grid_dep_wait();   // global memory from here on
+    // The plan reads only the sequence lengths, which no kernel of a decode step
+    // writes: it is made, down to this partition's first segment, before
+    // waiting for the kernel ahead on the stream (which produces q).
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, -1);
@@ -1214,16 +1216,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int64_t ts = (part < c.parts) ? part_start(part, N, c.parts) : N;
         const SeqCursor s = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, ts);
+        SegmentWalker w0;
+        w0.seq_lens = args.seq_lens;
+        w0.batch = args.batch;
+        w0.max_pages = args.max_pages;
+        w0.n_q = args.n_q;
+        w0.tile_tokens = TOK;
+        w0.N = N;
+        w0.P = c.parts;
+        w0.p = part;
+        w0.b = s.b;
+        w0.O = s.cost_off;
+        w0.S = s.slot_base;
+        w0.tile = (part < c.parts) ? part_start(part, N, c.parts) : 0;
+        w0.te = (part < c.parts) ? part_start(part + 1, N, c.parts) : 0;
+        const bool have0 = w0.next();
         if (lane == 0) {
-            misc->cur_b = s.b;
-            misc->cur_O = s.cost_off;
-            misc->cur_S = s.slot_base;
+            misc->cur_b = w0.b;
+            misc->cur_O = w0.O;
+            misc->cur_S = w0.S;
             misc->cur_N = N;
             misc->cur_P = c.parts;
+            misc->first_tile = w0.tile;
+            misc->first_slot = have0 ? w0.slot : 0;
+            misc->first_b = have0 ? w0.seg_b : -1;
+            misc->first_L = have0 ? w0.L : 0;
+            misc->first_t_begin = have0 ? static_cast<int32_t>(w0.t_begin) : 0;
+            misc->first_t_end = have0 ? static_cast<int32_t>(w0.t_end) : 0;
+            if (have0)   // the first page numbers, for the producer (a hint: L2 only)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                    args.block_table + static_cast<int64_t>(w0.seg_b) * args.max_pages + 2 * w0.t_begin));
             ptx::prefetch_tensormap(&map_ckv);
             ptx::prefetch_tensormap(&map_kr);
         }
     }
+    ptx::grid_dep_wait();   // other global memory from here on
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -1241,12 +1268,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     walk.b = misc->cur_b;
     walk.O = misc->cur_O;
     walk.S = misc->cur_S;
-    if (part < walk.P) {
-        walk.tile = part_start(part, walk.N, walk.P);
-        walk.te = part_start(part + 1, walk.N, walk.P);
-    } else {
-        walk.tile = walk.te = 0;   // idle partition
-    }
+    walk.te = (part < walk.P) ? part_start(part + 1, walk.N, walk.P) : 0;   // 0: idle partition
+    walk.tile = misc->first_tile;
+    walk.primed = misc->first_b >= 0;   // every role starts from the published first segment
+    walk.seg_b = misc->first_b;
+    walk.L = misc->first_L;
+    walk.t_begin = misc->first_t_begin;
+    walk.t_end = misc->first_t_end;
+    walk.slot = misc->first_slot;
 
     if (warp == 0) {
         if (ptx::elect_one()) {

@@ -155,13 +155,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t b = blockIdx.x;
     ptx::grid_dep_launch();
-    ptx::grid_dep_wait();   // the partials come from the kernel before
+    // the slot plan reads only the sequence lengths, which no kernel of a step
+    // writes: made before waiting for the kernel before
     if (warp == 0) {
         int64_t base, cnt;
         sequence_slots(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts, b,
                        &base, &cnt);
         if (lane == 0) { s_base = base; s_count = cnt; }
     }
+    ptx::grid_dep_wait();   // the partials come from the kernel before
     __syncthreads();
     const int r = blockIdx.y * 4 + warp;
     if (r >= a.rows) return;
@@ -499,6 +501,12 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
             ptx::tma_load_3d(w_s + kb * 16384u + 8192u, &map_w, wfull, 64, k0, h);
         }
     }
+    // the slots of the tile's sequences: the plan reads only the sequence
+    // lengths, which no kernel of a step writes, so it is made before the wait
+    const int32_t b_lo = t0 / a.n_q, b_hi = (t0 + nt - 1) / a.n_q;   // at most NT sequences
+    if (warp == 0)
+        sequence_slots_range(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts,
+                             b_lo, b_hi, seq_base, seq_cnt);
     ptx::grid_dep_wait();   // other global memory from here on
     if (warp == 1) {
         ptx::tmem_alloc<1>(ptx::smem_u32(tmem_slot), tcols);
@@ -510,14 +518,9 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     volatile int32_t *abort_v = abort_flag;
 
-    // ---- merge, phase 1: the slots of the tile's sequences (one warp, one
-    // pass), then eight threads per token find L and the weights exp(lse_s - L)
-    // with the same arithmetic and the same addition tree as combine_kernel
-    const int32_t b_lo = t0 / a.n_q, b_hi = (t0 + nt - 1) / a.n_q;   // at most NT sequences
-    if (warp == 0)
-        sequence_slots_range(a.seq_lens, a.batch, a.max_pages, a.n_q, a.tile_tokens, a.num_parts,
-                             b_lo, b_hi, seq_base, seq_cnt);
-    __syncthreads();
+    // ---- merge, phase 1: eight threads per token find L and the weights
+    // exp(lse_s - L) with the same arithmetic and the same addition tree as
+    // combine_kernel (the slots were found above; the barrier above publishes them)
     for (int tt = threadIdx.x >> 3; tt < NT; tt += 16) {
         const int sub = threadIdx.x & 7;
         const bool live = tt < nt;
