@@ -593,15 +593,16 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
             }
             // eight independent partial maxima / sums: one warp per SM sub-partition runs
             // this, so a single 128-long dependent chain would expose its full latency
+            // (three-input max: two new keys per instruction)
             float m8[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) m8[q] = v[q];
+            for (int q = 0; q < 8; ++q) m8[q] = fmaxf(v[q], v[8 + q]);
 #pragma unroll
-            for (int j = 8; j < TOK; j += 8)
+            for (int j = 16; j < TOK; j += 16)
 #pragma unroll
-                for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], v[j + q]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                for (int q = 0; q < 8; ++q) m8[q] = fmax3(m8[q], v[j + q], v[j + 8 + q]);
+            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                   fmaxf(m8[6], m8[7]));
             float alpha = 1.f;
             if (mx > -INFINITY &&
                 (m_run == -INFINITY || (mx - m_run) * args.scale_log2 > kRescaleThreshold)) {
@@ -609,15 +610,23 @@ __global__ void __launch_bounds__(pfa::THREADS, 1)
                 m_run = mx;
             }
             const float mb = (m_run == -INFINITY) ? 0.f : m_run * args.scale_log2;
-            float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            // the scaling and the eight partial sums two lanes per instruction
+            // (fma / add .f32x2): the loop is bound by issue slots, not by MUFU
+            const float2 sc2 = make_float2(args.scale_log2, args.scale_log2);
+            const float2 nmb2 = make_float2(-mb, -mb);
+            float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
 #pragma unroll
             for (int j = 0; j < TOK; j += 8)
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    v[j + q] = exp2f(fmaf(v[j + q], args.scale_log2, -mb));
-                    s8[q] += v[j + q];
+                for (int q = 0; q < 8; q += 2) {
+                    const float2 x = fma_f32x2(make_float2(v[j + q], v[j + q + 1]), sc2, nmb2);
+                    v[j + q] = exp2f(x.x);
+                    v[j + q + 1] = exp2f(x.y);
+                    s2[q >> 1] = add_f32x2(s2[q >> 1], make_float2(v[j + q], v[j + q + 1]));
                 }
-            const float psum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+            const float psum = ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) +
+                               ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y));
             l_run = fmaf(l_run, alpha, psum);
             const bool need = (k > 0) && (alpha != 1.f);
             if (__any_sync(0xffffffffu, need)) {
