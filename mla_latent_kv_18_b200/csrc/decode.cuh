@@ -477,8 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
             ptx::prefetch_tensormap(&map_ckv32);
             ptx::prefetch_tensormap(&map_ckv64);
             ptx::prefetch_tensormap(&map_kr32);
-            ptx::prefetch_tensormap(&map_q);
             if (kFp8) ptx::prefetch_tensormap(&map_sc);
+            else ptx::prefetch_tensormap(&map_q);
         }
     }
     ptx::grid_dep_wait();   // other global memory from here on
@@ -525,9 +525,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
             const uint32_t tx = kFp8 ? 2 * (OWN * 128) : 2 * (qk ? STAGE_QK : STAGE_PV);
             int64_t k = 0;
             bool bad_page = false;
-            if (qk && walk.primed) {
+            if (!kFp8 && qk && walk.primed) {
                 // the first segment's Q: blocks 0..QT-1 to the staging area (the
-                // segment warps move them to tensor memory), the rest to their place
+                // segment warps move them to tensor memory), the rest to their place.
+                // (The E4M3 kernel loads it like any other segment's: at its
+                // 128-register cap the staged path made the dequantising warps spill.)
                 const uint32_t qbar = bar(&misc->q_tma);
                 ptx::mbar_arrive_expect_tx(qbar, NB * ROWS_CTA * 128);
                 for (int j = 0; j < NB; ++j)
@@ -550,7 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
                     if (use >= 1 && !wait_bounded(bar(&emptyb[s]), (use - 1) & 1, abort_flag,
                                                   args.timeout_ns))
                         break;
-                    if (!qk && k == 1 &&   // slot 1 held the first segment's staged Q
+                    if (!kFp8 && !qk && k == 1 &&   // slot 1 held the first segment's staged Q
                         !wait_bounded(bar(&misc->q_stage_free), 0, abort_flag, args.timeout_ns))
                         break;
                     const uint32_t fb = (rank == 0) ? bar(&fullb[s]) : leader_bar(&fullb[s]);
@@ -879,7 +881,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         int64_t k = 0;
         int64_t g = 0;
         bool have = walk.next();
-        if (have) load_q_staged();
+        if (have) {
+            if constexpr (kFp8) load_q(walk.seg_b);
+            else load_q_staged();
+        }
         while (have && !*abort_flag) {
             const int64_t slot = walk.slot;
             const int64_t kl = k + (walk.t_end - walk.t_begin) - 1;   // the segment's last tile
