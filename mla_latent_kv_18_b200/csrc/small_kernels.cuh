@@ -360,6 +360,31 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
             }
             ptx::mma_commit(ptx::smem_u32(done));
         }
+    } else if (a.rope && blockIdx.y == 0) {
+        // warps 2 and 3, idle until the epilogue: q_r copied pair by pair
+        // while the MMA runs; with positions, pair (2p, 2p + 1) turns by
+        // pos * theta^(-2p / d_rope) ("MHA2MLA" page §3.2): angle and its
+        // reduction to [-pi, pi] in fp64 (large positions keep their phase),
+        // the rotation itself in fp32, the result rounded to bf16
+        const int half_r = a.d_rope / 2;
+        const int nt_r = min(a.NT, a.T - t0);
+        for (int i = threadIdx.x - 64; i < nt_r * half_r; i += 64) {
+            const int t = i / half_r, pr = i - t * half_r;
+            const int64_t src = (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + 2 * pr;
+            const int64_t dst = (static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + a.n_cols + 2 * pr;
+            const __nv_bfloat16 x0 = a.rope[src], x1 = a.rope[src + 1];
+            if (a.positions) {
+                int32_t pos = a.positions[t0 + t];
+                if (pos < 0) {
+                    record_error(kErrDeviceBounds);
+                    pos = 0;
+                }
+                rope_rotate_pair(x0, x1, pos, pr, a.d_rope, a.log_theta, &a.out[dst], &a.out[dst + 1]);
+            } else {
+                a.out[dst] = x0;
+                a.out[dst + 1] = x1;
+            }
+        }
     }
     // epilogue: TMEM lane = output column m0 + 32*warp + lane, column = token
     const bool ok = wait_bounded(ptx::smem_u32(done), 0, abort_v, a.timeout_ns);
@@ -379,30 +404,6 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
                         a.out[(static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + col] =
                             __float2bfloat16_rn(__uint_as_float(v[j]));
                 }
-            }
-        }
-    }
-    if (a.rope && blockIdx.y == 0) {
-        // q_r copied pair by pair; with positions, pair (2p, 2p + 1) turns by
-        // pos * theta^(-2p / d_rope) ("MHA2MLA" page §3.2): angle and its
-        // reduction to [-pi, pi] in fp64 (large positions keep their phase),
-        // the rotation itself in fp32, the result rounded to bf16
-        const int half_r = a.d_rope / 2;
-        for (int i = threadIdx.x; i < nt * half_r; i += 128) {
-            const int t = i / half_r, pr = i - t * half_r;
-            const int64_t src = (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + 2 * pr;
-            const int64_t dst = (static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + a.n_cols + 2 * pr;
-            const __nv_bfloat16 x0 = a.rope[src], x1 = a.rope[src + 1];
-            if (a.positions) {
-                int32_t pos = a.positions[t0 + t];
-                if (pos < 0) {
-                    record_error(kErrDeviceBounds);
-                    pos = 0;
-                }
-                rope_rotate_pair(x0, x1, pos, pr, a.d_rope, a.log_theta, &a.out[dst], &a.out[dst + 1]);
-            } else {
-                a.out[dst] = x0;
-                a.out[dst + 1] = x1;
             }
         }
     }
