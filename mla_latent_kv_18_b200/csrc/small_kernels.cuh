@@ -248,6 +248,17 @@ __device__ __forceinline__ void rope_rotate_pair(__nv_bfloat16 x0, __nv_bfloat16
     *y1 = __float2bfloat16_rn(f0 * sn + f1 * c);
 }
 
+// rope_rotate_pair on a packed bf16x2 word (x0 in the low half). Out of line: its
+// fp64 angle reduction is large, and the copy loop that calls it is unrolled.
+__device__ __noinline__ uint32_t rope_rotate_word(uint32_t w, int32_t pos, int pr, int d_rope,
+                                                  double log_theta) {
+    __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+    __nv_bfloat16 y0, y1;
+    rope_rotate_pair(x.x, x.y, pos, pr, d_rope, log_theta, &y0, &y1);
+    const __nv_bfloat162 y = __halves2bfloat162(y0, y1);
+    return *reinterpret_cast<const uint32_t *>(&y);
+}
+
 struct ProjArgs {
     __nv_bfloat16 *out;          // [T, H, out_stride]
     const __nv_bfloat16 *rope;   // [T, H, d_rope] or null (absorb-in copies q_r)
@@ -361,28 +372,45 @@ __global__ void __launch_bounds__(128) proj_tc_kernel(const __grid_constant__ CU
             ptx::mma_commit(ptx::smem_u32(done));
         }
     } else if (a.rope && blockIdx.y == 0) {
-        // warps 2 and 3, idle until the epilogue: q_r copied pair by pair
-        // while the MMA runs; with positions, pair (2p, 2p + 1) turns by
+        // warps 2 and 3, idle until the epilogue: q_r copied while the MMA runs,
+        // 16 bytes (four pairs) at a time, every load of a round issued before
+        // its stores (q_r rows and the q_out tail are 16-byte aligned: d_rope and
+        // d_latent are multiples of 8). With positions, pair (2p, 2p + 1) turns by
         // pos * theta^(-2p / d_rope) ("MHA2MLA" page §3.2): angle and its
-        // reduction to [-pi, pi] in fp64 (large positions keep their phase),
-        // the rotation itself in fp32, the result rounded to bf16
-        const int half_r = a.d_rope / 2;
-        const int nt_r = min(a.NT, a.T - t0);
-        for (int i = threadIdx.x - 64; i < nt_r * half_r; i += 64) {
-            const int t = i / half_r, pr = i - t * half_r;
-            const int64_t src = (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + 2 * pr;
-            const int64_t dst = (static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride + a.n_cols + 2 * pr;
-            const __nv_bfloat16 x0 = a.rope[src], x1 = a.rope[src + 1];
-            if (a.positions) {
-                int32_t pos = a.positions[t0 + t];
-                if (pos < 0) {
-                    record_error(kErrDeviceBounds);
-                    pos = 0;
+        // reduction to [-pi, pi] in fp64 (large positions keep their phase), the
+        // rotation itself in fp32, the result rounded to bf16
+        const int n8 = a.d_rope / 8;                   // 16-byte chunks per (token, head) row
+        const int items = min(a.NT, a.T - t0) * n8;
+        constexpr int U = 8;                           // chunks in flight per thread
+        for (int i0 = threadIdx.x - 64; i0 < items; i0 += 64 * U) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + 64 * u;
+                if (i < items) {
+                    const int t = i / n8, c8 = i - t * n8;
+                    v[u] = *reinterpret_cast<const uint4 *>(
+                        a.rope + (static_cast<int64_t>(t0 + t) * a.H + h) * a.d_rope + 8 * c8);
                 }
-                rope_rotate_pair(x0, x1, pos, pr, a.d_rope, a.log_theta, &a.out[dst], &a.out[dst + 1]);
-            } else {
-                a.out[dst] = x0;
-                a.out[dst + 1] = x1;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + 64 * u;
+                if (i >= items) continue;
+                const int t = i / n8, c8 = i - t * n8;
+                if (a.positions) {
+                    int32_t pos = a.positions[t0 + t];
+                    if (pos < 0) {
+                        record_error(kErrDeviceBounds);
+                        pos = 0;
+                    }
+                    v[u].x = rope_rotate_word(v[u].x, pos, 4 * c8 + 0, a.d_rope, a.log_theta);
+                    v[u].y = rope_rotate_word(v[u].y, pos, 4 * c8 + 1, a.d_rope, a.log_theta);
+                    v[u].z = rope_rotate_word(v[u].z, pos, 4 * c8 + 2, a.d_rope, a.log_theta);
+                    v[u].w = rope_rotate_word(v[u].w, pos, 4 * c8 + 3, a.d_rope, a.log_theta);
+                }
+                *reinterpret_cast<uint4 *>(a.out + (static_cast<int64_t>(t0 + t) * a.H + h) * a.out_stride +
+                                           a.n_cols + 8 * c8) = v[u];
             }
         }
     }
