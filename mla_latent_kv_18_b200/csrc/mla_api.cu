@@ -65,8 +65,14 @@ constexpr int32_t kGatherMaxWidth = 512;
 struct DeviceState {
     std::once_flag once;
     mla_status status = MLA_OK;
+    int sms = 0;   // multiprocessor count
 };
 DeviceState g_dev[kMaxDevices];
+
+int device_sms() {   // after device_ready() succeeded
+    int dev = 0;
+    return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) ? g_dev[dev].sms : 0;
+}
 
 mla_status device_ready() {
     int dev = 0;
@@ -77,6 +83,7 @@ mla_status device_ready() {
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { st.status = MLA_ERR_CUDA; return; }
         if (prop.major != 10 || prop.minor != 0) { st.status = MLA_ERR_UNSUPPORTED; return; }
+        st.sms = prop.multiProcessorCount;
         if (cudaFuncSetAttribute(mla::decode_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::pair::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -92,7 +99,7 @@ mla_status device_ready() {
             cudaFuncSetAttribute(mla::gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  64 * kGatherMaxWidth * 2) != cudaSuccess ||
             cudaFuncSetAttribute(mla::combine_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 mla::co_smem_bytes(128, mla::kCoMaxNT)) != cudaSuccess ||
+                                 mla::co_smem_bytes(128, mla::kCoMaxNT, mla::kCoMaxSlots)) != cudaSuccess ||
             cudaFuncSetAttribute(mla::decompress_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  mla::dkv::SMEM_BYTES) != cudaSuccess ||
@@ -708,7 +715,16 @@ mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(dims->num_heads * KS), static_cast<unsigned>((T + NT - 1) / NT));
     cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = mla::co_smem_bytes(KC, NT);
+    a.max_slots = num_parts + 1;   // < kCoMaxSlots + 1 (checked above)
+    static_assert(16 * 128 * 4 <= 16384, "the partial D tile fits in one K block of W_UV rows");
+    // Five CTAs fit on an SM: a grid larger than one wave at four per SM takes five
+    // (fewer waves); one that fits is kept at four, spread over more SMs (the merge
+    // is bound by each SM's load bandwidth), by requesting more than a fifth of
+    // the SM's shared memory.
+    uint32_t smem = mla::co_smem_bytes(KC, NT, a.max_slots);
+    const int64_t grid = static_cast<int64_t>(dims->num_heads) * KS * ((T + NT - 1) / NT);
+    if (grid <= 4 * static_cast<int64_t>(device_sms())) smem = std::max(smem, mla::kCoFourPerSmSmem);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;

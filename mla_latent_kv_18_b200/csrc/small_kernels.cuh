@@ -468,15 +468,20 @@ struct CombineOutArgs {
     float *lse_out;          // [T, H] or null
     int64_t timeout_ns;
     int32_t batch, max_pages, n_q, H, rows, d_c, d_v, tile_tokens, num_parts, T, NT, KS;
+    int32_t max_slots;       // capacity of the per-token weight rows: num_parts + 1
 };
 
 constexpr int kCoMaxNT = 64;
 constexpr int kCoMaxSlots = 160;   // partial slots per sequence (num_parts + 1 at most)
-__host__ __device__ constexpr uint32_t co_smem_bytes(int KC, int NT) {
+// Shared memory of a combine_out_kernel CTA. The partial D tile of the K-split
+// ([t][col] fp32, NT * 512 bytes) reuses the W_UV rows once the MMA has read
+// them, and the weight rows hold max_slots entries, so that five CTAs fit on an
+// SM (the grid has H * KS CTAs per 16 tokens).
+constexpr uint32_t kCoFourPerSmSmem = 49152;   // above a fifth of the SM's 228 KB, within a quarter
+__host__ __device__ constexpr uint32_t co_smem_bytes(int KC, int NT, int max_slots) {
     return static_cast<uint32_t>(KC / 64) * 16384u            // W_UV rows: two 64-column atoms per K block
            + static_cast<uint32_t>(KC / 64) * NT * 128u        // merged rows (bf16, K-major, swizzled)
-           + static_cast<uint32_t>(NT) * 128u * 4u             // partial D tile [t][col] fp32
-           + static_cast<uint32_t>(NT) * kCoMaxSlots * 4u      // merge weights [t][slot]
+           + static_cast<uint32_t>(NT) * max_slots * 4u        // merge weights [t][slot]
            + static_cast<uint32_t>(NT) * 16u                   // per token: first slot, count, row
            + static_cast<uint32_t>(NT) * 16u                   // per sequence: first slot, count
            + 128u /* barriers */ + 1024u /* alignment */;
@@ -497,9 +502,10 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     const int nt = min(NT, a.T - t0);
     const uint32_t w_s = base;
     const uint32_t x_s = w_s + KB * 16384u;
-    const uint32_t part_s = x_s + KB * NT * 128u;
-    const uint32_t wts_s = part_s + NT * 128u * 4u;
-    const uint32_t tok_s = wts_s + NT * kCoMaxSlots * 4u;
+    const uint32_t part_s = w_s;   // the partial D tile, once the MMA has read the W_UV rows
+    const uint32_t wts_s = x_s + KB * NT * 128u;
+    const int MS = a.max_slots;
+    const uint32_t tok_s = wts_s + NT * MS * 4u;
     const uint32_t seq_s = tok_s + NT * 16u;
     const uint32_t bar_s = seq_s + NT * 16u;
     int64_t *seq_base = reinterpret_cast<int64_t *>(co_smem_raw + (seq_s - raw_base));
@@ -594,15 +600,15 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
         const float L = (m > -INFINITY) ? m + __logf(z) : -INFINITY;
         if (live && a.lse_out && q == 0 && sub == 0)
             a.lse_out[static_cast<int64_t>(t0 + tt) * a.H + h] = L;
-        if (m == -INFINITY || cnt > kCoMaxSlots) cnt = 0;   // nothing to merge (host caps the slots)
+        if (m == -INFINITY || cnt > MS) cnt = 0;   // nothing to merge (the host caps the slots)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int s = sub + 8 * j;
-            if (s < cnt) wts[tt * kCoMaxSlots + s] = (lv[j] > -INFINITY) ? __expf(lv[j] - L) : 0.f;
+            if (s < cnt) wts[tt * MS + s] = (lv[j] > -INFINITY) ? __expf(lv[j] - L) : 0.f;
         }
         for (int s = sub + 32; s < cnt; s += 8) {
             const float ls = lse_r[static_cast<int64_t>(s) * a.rows];
-            wts[tt * kCoMaxSlots + s] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
+            wts[tt * MS + s] = (ls > -INFINITY) ? __expf(ls - L) : 0.f;
         }
         if (sub == 0) {
             tok_base[tt] = sbase;
@@ -645,7 +651,7 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
                         const bool on = s + e < cnt_i[u];
                         v[u][e] = on ? *reinterpret_cast<const float4 *>(src[u] + (s + e) * slot_stride)
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                        w[u][e] = on ? wts[tt_i[u] * kCoMaxSlots + s + e] : 0.f;
+                        w[u][e] = on ? wts[tt_i[u] * MS + s + e] : 0.f;
                     }
 #pragma unroll
                 for (int u = 0; u < IT; ++u)
