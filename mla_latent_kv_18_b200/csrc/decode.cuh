@@ -430,9 +430,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kPairThreadsF
         ptx::tmem_relinquish<2>();
     }
     ptx::grid_dep_launch();
-    // The plan reads only the sequence lengths, which no kernel of a decode step
-    // writes (the kernel ahead on the stream produces q): it is made, down to
-    // this partition's first segment, before waiting for that kernel.
+    // The plan reads only the sequence lengths and the block table, which no
+    // kernel of a decode step writes (the kernel ahead on the stream produces
+    // q): it is made, down to this partition's first segment and that
+    // segment's first page ids, before waiting for that kernel.
     if (warp == 0) {
         const SeqCursor c = find_sequence(args.seq_lens, args.batch, args.max_pages, args.n_q, TOK,
                                           P, -1);
