@@ -685,9 +685,15 @@ mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
     const int64_t T64 = static_cast<int64_t>(batch) * dims->n_q;
     if (T64 > (int64_t(1) << 30)) return MLA_ERR_UNSUPPORTED;
     const int32_t T = static_cast<int32_t>(T64);
-    const int32_t NT = 16;   // tokens per CTA: the smallest MMA N, for the most CTAs (W_UV re-reads hit L2)
     const int32_t KS = dc >= 256 ? dc / 128 : 1;
     const int32_t KC = dc / KS;
+    // Tokens per CTA: 16 (the smallest MMA N, the most CTAs; W_UV re-reads hit L2)
+    // while the grid fits in one wave of five CTAs per SM; a larger one takes 32
+    // (half the CTAs and waves, each W_UV slice read half as often).
+    const int32_t NT =
+        (static_cast<int64_t>(dims->num_heads) * KS * ((T + 15) / 16) > 5 * static_cast<int64_t>(device_sms()))
+            ? 32
+            : 16;
     CUtensorMap mw;
     if ((st = map_3d(&mw, w_uv, dims->d_v, dc, dims->num_heads, uint64_t(dims->d_v) * 2,
                      uint64_t(dc) * dims->d_v * 2, 64, 64, 1)) != MLA_OK)
@@ -716,7 +722,7 @@ mla_status mla_combine_absorb_out(const mla_dims *dims, const void *workspace,
     cfg.gridDim = dim3(static_cast<unsigned>(dims->num_heads * KS), static_cast<unsigned>((T + NT - 1) / NT));
     cfg.blockDim = dim3(128);
     a.max_slots = num_parts + 1;   // < kCoMaxSlots + 1 (checked above)
-    static_assert(16 * 128 * 4 <= 16384, "the partial D tile fits in one K block of W_UV rows");
+    static_assert(32 * 128 * 4 <= 16384, "the partial D tile fits in one K block of W_UV rows");
     // Five CTAs fit on an SM: a grid larger than one wave at four per SM takes five
     // (fewer waves); one that fits is kept at four, spread over more SMs (the merge
     // is bound by each SM's load bandwidth), by requesting more than a fifth of

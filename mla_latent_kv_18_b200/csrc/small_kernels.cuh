@@ -476,7 +476,7 @@ constexpr int kCoMaxSlots = 160;   // partial slots per sequence (num_parts + 1 
 // Shared memory of a combine_out_kernel CTA. The partial D tile of the K-split
 // ([t][col] fp32, NT * 512 bytes) reuses the W_UV rows once the MMA has read
 // them, and the weight rows hold max_slots entries, so that five CTAs fit on an
-// SM (the grid has H * KS CTAs per 16 tokens).
+// SM (the grid has H * KS CTAs per 16 or 32 tokens).
 constexpr uint32_t kCoFourPerSmSmem = 49152;   // above a fifth of the SM's 228 KB, within a quarter
 __host__ __device__ constexpr uint32_t co_smem_bytes(int KC, int NT, int max_slots) {
     return static_cast<uint32_t>(KC / 64) * 16384u            // W_UV rows: two 64-column atoms per K block
@@ -621,7 +621,7 @@ __global__ void __launch_bounds__(128) combine_out_kernel(const __grid_constant_
     // issued together; slots are added in order, as in combine_kernel
     {
         const int chunks = KC / 4;
-        constexpr int IT = 4;   // items per thread (NT * chunks <= 16 * 32 = 512 = 4 x 128)
+        constexpr int IT = 4;   // items per thread and round (NT * chunks / 512 rounds)
         const int64_t slot_stride = static_cast<int64_t>(a.rows) * a.d_c;
         for (int i0 = threadIdx.x; i0 < NT * chunks; i0 += IT * 128) {
             float4 acc[IT];

@@ -156,7 +156,17 @@ def test_parity_dsv3(api):
 
 
 def test_parity_ragged(api):
-    _parity(api, workload("ragged"), 8)
+    r, inp = _parity(api, workload("ragged"), 8)
+    # the fused combine + absorb-out at 64 tokens (a grid of more than one wave: 32
+    # tokens per CTA) on the same full-size partials
+    d = to_device(inp, "cuda")
+    lse = torch.empty_like(r["lse"])
+    fused = api.combine_absorb_out(r["ws"], d["seq_lens"], d["block_table"].shape[1], r["dims"],
+                                   r["num_parts"], d["w_uv"], lse_out=lse)
+    torch.cuda.synchronize()
+    assert api.get_device_error() == 0
+    assert torch.equal(lse, r["lse"])
+    _check_one_ulp(_f64(fused), _f64(r["out"]), "ragged: fused vs unfused")
 
 
 def test_parity_retrofit(api):
@@ -354,6 +364,7 @@ def test_gather_bad_page_id_sets_device_error(api):
 
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("dsv3", dict(batch=4, seq_len=3000)),
                                      ("dsv3", dict(batch=80, heads=16, seq_len=200)),
+                                     ("dsv3", dict(batch=48, heads=128, seq_len=300)),   # 32 tokens per CTA, ragged tail
                                      ("ragged", dict(batch=6, heads=128, ragged=(64, 4000))),
                                      ("retrofit", dict(batch=9, seq_len=700))])
 def test_fused_combine_absorb_out(api, name, kw):
