@@ -180,6 +180,13 @@ def test_argument_validation_without_launch(b):
     assert lib.mla_decode_splitkv(ctypes.byref(d), fake, ctypes.byref(good), ctypes.byref(good),
                                   1, fake, 1, fake, 2, 1, ctypes.c_void_p(0x10010), ws_bytes,
                                   null) == 1                # workspace not 256-byte aligned
+    # the fused combine holds at most num_parts + 1 <= 160 slots per sequence in its
+    # weight rows: 160 partitions are refused, 159 pass that check (and stop here at
+    # the null workspace, before any device call)
+    assert lib.mla_combine_absorb_out(ctypes.byref(d), null, 0, fake, 1, 2, 160, fake, fake, null,
+                                      null) == 2
+    assert lib.mla_combine_absorb_out(ctypes.byref(d), null, 0, fake, 1, 2, 159, fake, fake, null,
+                                      null) == 1
     assert lib.mla_debug_wait_timeout(0, null) == 1
 
 
